@@ -1,0 +1,533 @@
+#!/usr/bin/env python
+"""Benchmark of the Gemma-4-26B-A4B MoE feed-forward block on B200.
+
+One "step" is one pass of the block (router, top-k, permutation, gate|up and
+down grouped GEMMs, shared MLP, combine) over one batch of T tokens, through
+the library's C ABI. Default workload: the decode-sized block, T = 64 tokens.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload decode|tiny|prefill|skewed]
+  python bench.py --impl reference ...   # the CPU oracle on the same workload
+
+N > 1 (torchrun) runs N independent replicas, one per GPU: tokens are
+independent in the block, so each rank processes its own batch with no
+data-path collective (weak scaling). Timing is on the device with CUDA events,
+bracketed by a barrier and a synchronize, max over ranks.
+
+Prints ONE JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+D, E, F, S, K_TOP = 2816, 128, 704, 2112, 8
+BYTES_PER_EXPERT = 3 * D * F * 2  # gate, up, down bf16
+SHARED_BYTES = 3 * D * S * 2
+ROUTER_BYTES = D * E * 2
+FLOP_PER_TOKEN_GEMM = 2 * K_TOP * 3 * D * F + 2 * 3 * D * S  # tensor-core work
+FLOP_PER_TOKEN = FLOP_PER_TOKEN_GEMM + 2 * D * E
+
+WORKLOADS = {
+    "tiny": dict(T=8, bias=False, bound="hbm", desc="Gemma-4-26B-A4B MoE block, T=8 tokens, bf16"),
+    "decode": dict(T=64, bias=False, bound="hbm", desc="Gemma-4-26B-A4B MoE block, decode-sized T=64 tokens, bf16"),
+    "prefill": dict(T=4096, bias=False, bound="tensor", desc="Gemma-4-26B-A4B MoE block, prefill-sized T=4096, bf16"),
+    "skewed": dict(
+        T=16384, bias=True, bound="tensor", desc="Gemma-4-26B-A4B MoE block, T=16384, Zipf(1.1) router bias, bf16"
+    ),
+}
+METRIC = "MoE-block tokens/s"
+
+NVML_REASONS = {
+    0x1: "gpu_idle",
+    0x2: "applications_clocks_setting",
+    0x4: "sw_power_cap",
+    0x8: "hw_slowdown",
+    0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------ distributed
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max over ranks (a barrier + one all-reduce); identity at world 1."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def aggregate(tokens_per_rank: int, steps: int, ms_max: float, world: int) -> dict:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    total_tokens = tokens_per_rank * steps * world
+    return {"value": total_tokens / (ms_max / 1e3), "ms_per_step": ms_max / steps}
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: report no clocks
+            self._nvml = None
+
+    def _reasons_now(self):
+        n = self._nvml
+        fn = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or n.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self._h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons_now())
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def report(self):
+        if not self._nvml:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml_unavailable"], "samples": 0}
+        names = [v for k, v in NVML_REASONS.items() if self.reasons & k and v != "gpu_idle"]
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": names,
+            "samples": len(self.samples),
+        }
+
+
+# ----------------------------------------------------------------- peaks
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_experts_transformer_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    ent = table.get(f"{kernel}@{workload}")
+    if not ent or ent.get("csrc") != csrc_digest():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------- algorithmics
+
+
+def algorithmic(kernel: str, T: int, touched: int, cnt: np.ndarray):
+    """Algorithmic bytes and FLOPs of one launch of a kernel (each operand and
+    result once)."""
+    R = T * K_TOP
+    if kernel == "grouped_gemm_gateup":
+        byts = touched * 2 * D * F * 2 + 2 * D * S * 2 + R * D * 2 + T * D * 2 + R * F * 2 + T * S * 2
+        flops = 2 * 2 * D * (R * F + T * S)
+    elif kernel == "grouped_gemm_down":
+        byts = touched * F * D * 2 + S * D * 2 + R * F * 2 + T * S * 2 + R * D * 2 + T * D * 4
+        flops = 2 * D * (R * F + T * S)
+    elif kernel == "gather_rows":
+        byts = T * D * 2 + R * D * 2
+        flops = 0
+    elif kernel == "combine":
+        byts = R * D * 2 + T * D * 4 + T * D * 2
+        flops = 2 * R * D
+    elif kernel == "router_logits":
+        byts = T * D * 2 + D * E * 2
+        flops = 2 * T * D * E
+    else:
+        byts, flops = 0, 0
+    return byts, flops
+
+
+# --------------------------------------------------------------- our arm
+
+
+def gen_weights_gpu(seed: int = 0, std: float = 0.02):
+    """Random-init weights of the published shapes, drawn on the GPU (seeded)."""
+    import torch
+
+    g = torch.Generator(device="cuda").manual_seed(seed)
+
+    def rnd(*shape, s=std):
+        return torch.empty(shape, dtype=torch.float32, device="cuda").normal_(0.0, s, generator=g).to(torch.bfloat16)
+
+    from mixture_experts_transformer_b200 import block, inputs
+
+    return block.DeviceWeights(
+        inputs.GEMMA4_26B_A4B,
+        rnd(D, E),
+        rnd(E, D, F),
+        rnd(E, D, F),
+        rnd(E, F, D),
+        rnd(D, S),
+        rnd(D, S),
+        rnd(S, D),
+    )
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from mixture_experts_transformer_b200 import binding as B
+    from mixture_experts_transformer_b200 import block, build, inputs
+
+    if rank == 0:
+        build.build()
+    barrier(world)
+    B.lib()
+    torch.cuda.set_device(local)
+    wl = WORKLOADS[args.workload]
+    T = wl["T"]
+    dw = gen_weights_gpu(seed=0)
+    gx = torch.Generator(device="cuda").manual_seed(1 + rank)
+    x = torch.empty((T, D), dtype=torch.float32, device="cuda").normal_(0.0, 1.0, generator=gx).to(torch.bfloat16)
+    bias = torch.from_numpy(inputs.zipf_router_bias()).cuda() if wl["bias"] else None
+    out = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    ws, _ = block.workspace_for(inputs.GEMMA4_26B_A4B, T)
+    stream = torch.cuda.current_stream()
+    p = B.make_params(T, x, *dw.args(), out, router_bias=bias, workspace=ws)
+
+    # routing statistics of this batch (outside the timed region)
+    dbg = block.forward(dw, x, router_bias=bias, debug=True, workspace=ws)
+    torch.cuda.synchronize()
+    cnt = dbg.cnt.cpu().numpy()
+    touched = int((cnt > 0).sum())
+    st = B.moe_get_device_status()
+    if st != B.MOE_OK:
+        raise RuntimeError(B.moe_status_string(st))
+
+    for _ in range(args.warmup):
+        B.check(B.moe_block_forward_ex(p, stream), "forward")
+    torch.cuda.synchronize()
+    launches_per_step = B.moe_last_launch_count()
+
+    # ---- timed region: device events, per-kernel events recorded live
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        B.moe_profile_begin()
+        e0.record(stream)
+        for _ in range(args.steps):
+            B.check(B.moe_block_forward_ex(p, stream), "forward")
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_kernel = B.moe_profile_end()
+    barrier(world)
+    ms_local = e0.elapsed_time(e1)
+    ms = reduce_max(ms_local, world)
+    agg = aggregate(T, args.steps, ms, world)
+    st = B.moe_get_device_status()
+    if st != B.MOE_OK:
+        raise RuntimeError(B.moe_status_string(st))
+
+    # ---- end to end: host buffers through the C ABI, copies inside the timed region
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        B.check(B.moe_block_forward_hostio(p, x_host, out_host, stream), "hostio")
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        B.check(B.moe_block_forward_hostio(p, x_host, out_host, stream), "hostio")
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(t0.elapsed_time(t1), world)
+    barrier(world)
+    if not torch.equal(out_host, out.cpu()):
+        raise RuntimeError("host-buffer path disagrees with the device path")
+
+    if rank != 0:
+        return None
+
+    peaks = measured_peaks()
+    kernel_ms = {k: v[0] / v[1] for k, v in per_kernel.items()}
+    dominant = max(per_kernel, key=lambda k: per_kernel[k][0])
+    byts, flops = algorithmic(dominant, T, touched, cnt)
+    dom_ms = kernel_ms[dominant]
+    long_region = ms / 1e3 > 2.0
+    if wl["bound"] == "hbm":
+        achieved = byts / (dom_ms / 1e3) / 1e9
+        peak, unit, peak_name = peaks["hbm_gbs"], "GB/s", "hbm_gbs"
+    else:
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        peak, unit, peak_name = peaks[key], "TFLOP/s", key
+    traffic = ncu_traffic(dominant, args.workload)
+    step_ms = agg["ms_per_step"]
+    weight_bytes = touched * BYTES_PER_EXPERT + SHARED_BYTES + ROUTER_BYTES
+    block_roof = {
+        "hbm_touched_weights_gbs": weight_bytes / (step_ms / 1e3) / 1e9,
+        "hbm_frac": weight_bytes / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "tensor_tflops": T * FLOP_PER_TOKEN_GEMM / (step_ms / 1e3) / 1e12,
+        "tensor_frac": T * FLOP_PER_TOKEN_GEMM / (step_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "touched_experts": touched,
+    }
+    res = {
+        "metric": METRIC,
+        "value": agg["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, x ~ N(0,1)",
+        "config": {
+            "workload": wl["desc"],
+            "tokens_per_gpu": T,
+            "global_batch": T * world,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (1.5 GB of expert weights per step)",
+            "router_bias": "zipf(1.1)" if wl["bias"] else None,
+        },
+        "roofline": {
+            "bound": wl["bound"],
+            "kernel": dominant,
+            "achieved": achieved,
+            "peak": peak,
+            "peak_source": f"{peaks['source']} {peak_name}",
+            "unit": unit,
+            "frac": achieved / peak,
+            "traffic": traffic,
+            "algorithmic_bytes": byts,
+            "algorithmic_flops": flops,
+            "kernel_ms": dom_ms,
+        },
+        "block_roofline": block_roof,
+        "kernels_ms_per_launch": kernel_ms,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {
+            "value": T * args.steps * world / (e2e_ms / 1e3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": T * D * 2,
+            "d2h_bytes_per_step": T * D * 2,
+        },
+        "clocks": clocks.report(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(dw, x, bias, T, budget_s=12.0)
+    return res
+
+
+# ----------------------------------------------------------- CPU oracle
+
+
+def _host_weights(dw):
+    from mixture_experts_transformer_b200 import inputs
+
+    def u16(t):
+        return t.cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+
+    return inputs.BlockWeights(*(u16(t) for t in dw.args()))
+
+
+def _oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) if threadpool_info() else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(dw, x, bias, T, budget_s=12.0, sample_tokens=None):
+    """The oracle as it stands, on a bounded sample of the same workload."""
+    from oracle import moe_oracle as mo
+
+    wh = _host_weights(dw)
+    xb = x.cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    b = None if bias is None else bias.cpu().numpy()
+    n = min(T, sample_tokens or 64)
+    xs = xb[:n]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        mo.moe_block(xs, wh.w_router, wh.wg, wh.wu, wh.wd, wh.sg, wh.su, wh.sd, top_k=K_TOP, bias=b)
+        done += n
+        if time.perf_counter() - t0 > budget_s or done >= 64 * n:
+            break
+    el = time.perf_counter() - t0
+    return {
+        "value": done / el,
+        "unit": "tokens/s",
+        "cores": _oracle_cores(),
+        "kind": "oracle",
+        "sample": f"{done} tokens ({done // n} passes over the first {n} tokens of the batch), {el:.1f} s",
+    }
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle on our arm's workload, metric and unit (rank 0 only)."""
+    if rank != 0:
+        return None
+    import torch
+
+    from mixture_experts_transformer_b200 import inputs
+    from oracle import moe_oracle as mo
+
+    wl = WORKLOADS[args.workload]
+    T = wl["T"]
+    w = inputs.make_weights()
+    n = min(T, 8)
+    x = inputs.make_x(n)
+    bias = inputs.zipf_router_bias() if wl["bias"] else None
+    for _ in range(args.warmup):
+        mo.moe_block(x, w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd, bias=bias)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        mo.moe_block(x, w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd, bias=bias)
+    el = time.perf_counter() - t0
+    v = n * args.steps / el
+    cores = _oracle_cores()
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": v,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, x ~ N(0,1)",
+        "config": {"workload": wl["desc"], "tokens_per_gpu": T, "global_batch": T * world, "parallelism": "single"},
+        "cpu_baseline": {
+            "value": v,
+            "unit": "tokens/s",
+            "cores": cores,
+            "kind": "oracle",
+            "sample": f"each step: the first {n} of the workload's {T} tokens through the fp64 oracle",
+        },
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_ours(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

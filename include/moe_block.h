@@ -1,0 +1,222 @@
+/*
+ * moe_block.h - C ABI of a B200 (sm_100a) library for one Gemma-4-26B-A4B
+ * mixture-of-experts feed-forward block.
+ *
+ * What the block computes (the layer's statement on the pages):
+ *   - gm.nn.Gemma4_26B_A4B, class docstring and TransformerConfig: every layer
+ *     has "a MoE branch (128 experts, expert_dim=704)" and "a dense shared
+ *     MLP branch" of width 2112 (hidden_dim = moe_dense_hidden_dim), with
+ *     embed_dim 2816, num_experts 128, top_k_experts 8, dtype bfloat16;
+ *   - Gemma-4-26B-A4B model card: gating "softmax" over expert logits, 8
+ *     routed experts per token, "Selected expert weights are renormalized to
+ *     sum to 1", one always-on expert of width 2112, FFN activation "GeGLU
+ *     (tanh-approximate GELU)", no FFN biases;
+ *   - G4-MeroMero-26B-A4B-NVFP4 config.json: the NVFP4 format (below).
+ *
+ *   logits[t, e] = sum_d x[t, d] * W_router[d, e]  (+ router_bias[e])
+ *   idx[t, 0..k-1] = the k largest logits, largest first; equal logits: the
+ *                    lower expert index first
+ *   w[t, j]        = softmax over all experts, restricted to idx[t, .] and
+ *                    renormalised (= softmax of the k kept logits)
+ *   ffn(x; G, U, D) = (gelu_tanh(x G) * (x U)) D,
+ *                    gelu_tanh(z) = z/2 (1 + tanh(sqrt(2/pi)(z + 0.044715 z^3)))
+ *   out[t] = ffn(x[t]; Sg, Su, Sd) + sum_j w[t, j] ffn(x[t]; Wg[e], Wu[e], Wd[e]),
+ *            e = idx[t, j]
+ *
+ * Numerics: bf16 inputs, fp32 accumulation everywhere; the GeGLU hidden rows
+ * h and the routed experts' outputs y are rounded to bf16 between kernels; the
+ * shared branch stays fp32; out is the round-to-nearest-even bf16 of the fp32
+ * sum (s + w_0 y_0 + w_1 y_1 + ..., in slot order). Results are bitwise
+ * deterministic for a given device and input.
+ *
+ * Conventions for every call:
+ *   - all tensor pointers are DEVICE pointers, row-major, contiguous, 16-byte
+ *     aligned, owned by the caller; the library never frees caller memory;
+ *   - bf16 means IEEE bfloat16 bit patterns (uint16_t here);
+ *   - calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream): they validate on the host, enqueue kernels and return
+ *     without synchronising, except moe_get_device_status;
+ *   - T == 0 is a no-op returning MOE_OK; invalid arguments return an error
+ *     before anything is enqueued;
+ *   - the library needs sm_100 (B200); other devices get MOE_ERR_ARCH.
+ */
+#ifndef MOE_BLOCK_H
+#define MOE_BLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, unsupported dims, aliasing */
+  MOE_ERR_ALIGNMENT = 2,     /* a pointer is not 16-byte aligned */
+  MOE_ERR_ARCH = 3,          /* the current device is not sm_100 */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, allocation) */
+  MOE_ERR_WORKSPACE = 5,     /* caller workspace smaller than moe_workspace_bytes_ex */
+  MOE_ERR_DEVICE_TIMEOUT = 6 /* a kernel's bounded wait ran out (reported by moe_get_device_status) */
+} moe_status;
+
+/* Gemma-4-26B-A4B block constants (TransformerConfig of gm.nn.Gemma4_26B_A4B). */
+#define MOE_EMBED_DIM 2816
+#define MOE_NUM_EXPERTS 128
+#define MOE_EXPERT_DIM 704
+#define MOE_HIDDEN_DIM 2112
+#define MOE_TOP_K 8
+
+/*
+ * Full parameter set. Dims left 0 take the Gemma-4-26B-A4B values above.
+ * Supported dims: embed_dim, expert_dim, hidden_dim multiples of 64;
+ * num_experts a multiple of 8 and <= 128; 1 <= top_k_experts <= num_experts.
+ *
+ * Weights (bf16, row-major, exactly as given - no repacking):
+ *   w_router [embed_dim, num_experts]
+ *   wg, wu   [num_experts, embed_dim, expert_dim]   (gate, up)
+ *   wd       [num_experts, expert_dim, embed_dim]   (down)
+ *   sg, su   [embed_dim, hidden_dim]                (shared gate, up)
+ *   sd       [hidden_dim, embed_dim]                (shared down)
+ * x [T, embed_dim] bf16 in; out [T, embed_dim] bf16 out, written fully; out
+ * must not overlap x.
+ *
+ * Optional (NULL = absent):
+ *   router_bias [num_experts] fp32, added to the logits before the softmax;
+ *   workspace / workspace_bytes: caller scratch of at least
+ *     moe_workspace_bytes_ex(p) bytes, 256-byte aligned; without it the
+ *     library uses one cached allocation per device (grown on demand, kept
+ *     until process exit; calls on different streams then share it, so run
+ *     them one after another or give each its own workspace);
+ *   out_f32 [T, embed_dim] fp32: the pre-rounding output (out == RNE(out_f32));
+ *   idx_out [T, top_k] int32, w_out [T, top_k] fp32: the routing used;
+ *   cnt_out [num_experts] int32: tokens per expert.
+ */
+typedef struct moe_params {
+  int T;
+  int top_k_experts;
+  int embed_dim;
+  int num_experts;
+  int expert_dim;
+  int hidden_dim;
+  const void* x;
+  const void* w_router;
+  const float* router_bias;
+  const void* wg;
+  const void* wu;
+  const void* wd;
+  const void* sg;
+  const void* su;
+  const void* sd;
+  void* out;
+  float* out_f32;
+  int32_t* idx_out;
+  float* w_out;
+  int32_t* cnt_out;
+  void* workspace;
+  size_t workspace_bytes;
+} moe_params;
+
+/*
+ * Where the block's intermediates live inside a workspace (byte offsets from
+ * its start; a size of 0 means the buffer is unused). R = T * top_k routed
+ * rows, ordered expert by expert, tokens ascending within an expert.
+ *   x_perm [R, embed_dim] bf16   - x gathered into routed-row order
+ *   h      [R, expert_dim] bf16  - routed GeGLU hidden rows
+ *   y      [R, embed_dim] bf16   - routed expert outputs (unweighted)
+ *   hs     [T, hidden_dim] bf16  - shared GeGLU hidden rows
+ *   s      [T, embed_dim] fp32   - shared MLP output
+ *   idx [T, top_k] int32, w [T, top_k] fp32, cnt [E] int32, off [E + 1] int32,
+ *   row_of [T, top_k] int32 (routed row of each (token, slot)),
+ *   token_of [R] int32 (token of each routed row)
+ */
+typedef struct moe_ws_layout {
+  size_t total_bytes;
+  size_t x_perm, h, y, hs, s;
+  size_t idx, w, cnt, off, row_of, token_of;
+} moe_ws_layout;
+
+/* Bytes of workspace a call with these params needs (T, top_k and dims are read). */
+size_t moe_workspace_bytes_ex(const moe_params* p);
+/* Same for the Gemma-4-26B-A4B dims. */
+size_t moe_workspace_bytes(int T, int top_k);
+/* Fill *out with the workspace layout for these params; MOE_ERR_INVALID_ARG on bad dims. */
+moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out);
+
+/*
+ * The block forward pass at the Gemma-4-26B-A4B dims, top_k 8, no router
+ * bias, library-owned workspace. Pointers as in moe_params.
+ */
+moe_status moe_block_forward(const void* x, const void* w_router, const void* wg, const void* wu, const void* wd,
+                             const void* sg, const void* su, const void* sd, int T, void* out, void* stream);
+
+/* The block forward pass with every option (see moe_params). */
+moe_status moe_block_forward_ex(const moe_params* p, void* stream);
+
+/*
+ * Router only (the first step of the block): logits in fp32, top-k selection
+ * and renormalised softmax weights. Uses p->T, top_k_experts, embed_dim,
+ * num_experts, x, w_router, router_bias and the workspace fields;
+ * writes idx [T, top_k] int32 and w [T, top_k] fp32.
+ */
+moe_status moe_route(const moe_params* p, int32_t* idx, float* w, void* stream);
+
+/*
+ * Expert-major permutation of the (token, slot) assignments in idx
+ * [T, top_k] (values in [0, num_experts)): cnt [num_experts] tokens per
+ * expert, off [num_experts + 1] exclusive scan of cnt, row_of [T, top_k]
+ * routed row of each assignment, token_of [T * top_k] token of each row. Rows
+ * of expert e are off[e] .. off[e+1]-1 in ascending token order. Integer
+ * work, bit-exact. Uses p->T, top_k_experts, num_experts, workspace fields.
+ */
+moe_status moe_permute(const moe_params* p, const int32_t* idx, int32_t* cnt, int32_t* off, int32_t* row_of,
+                       int32_t* token_of, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the library's device error word
+ * on the current device. MOE_ERR_DEVICE_TIMEOUT if any kernel gave up a
+ * bounded wait since the last call (its outputs are then undefined);
+ * MOE_ERR_CUDA if the stream reports a CUDA error.
+ */
+moe_status moe_get_device_status(void* stream);
+
+/*
+ * Failure-path check: launch one small kernel that waits, bounded by
+ * timeout_us microseconds, on a barrier that nothing will complete. The wait
+ * runs out, the kernel records MOE_ERR_DEVICE_TIMEOUT in the device error
+ * word and returns; the context stays usable.
+ */
+moe_status moe_debug_timeout_probe(int timeout_us, void* stream);
+
+/*
+ * End-to-end variant of moe_block_forward_ex for callers whose activations
+ * live in host memory: enqueues the copy of x_host (T * embed_dim bf16) into
+ * the device buffer p->x, the forward pass, and the copy of p->out back into
+ * out_host, all on `stream`. Host buffers should be pinned for the copies to
+ * be asynchronous; the caller synchronises `stream` before reading out_host.
+ */
+moe_status moe_block_forward_hostio(const moe_params* p, const void* x_host, void* out_host, void* stream);
+
+/*
+ * Per-kernel timing. After moe_profile_begin(), every kernel this thread
+ * enqueues is bracketed by two CUDA events recorded on its stream.
+ * moe_profile_end() waits for those events, writes per kernel id the summed
+ * milliseconds and the number of launches into total_ms[0..n) and
+ * launches[0..n), stops recording and returns the number of kernel ids.
+ * moe_kernel_name(id) names a kernel id (NULL past the last one).
+ */
+moe_status moe_profile_begin(void);
+int moe_profile_end(float* total_ms, int* launches, int n);
+const char* moe_kernel_name(int id);
+
+/* Human-readable name of a status code. */
+const char* moe_status_string(moe_status s);
+
+/* Number of kernels the last forward call on this thread enqueued. */
+int moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_BLOCK_H */

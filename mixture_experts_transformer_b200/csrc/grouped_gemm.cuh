@@ -1,0 +1,328 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA. One launch runs up to two "problems" (the routed experts and the
+// shared MLP) as a single list of 128-row work tiles built on the device.
+//
+//   GATEUP: h[row, n] = gelu_tanh(A Bg)[row, n] * (A Bu)[row, n]   (bf16 out)
+//   DOWN:   y[row, n] = (A Bd)[row, n]                            (bf16 or fp32 out)
+//
+// A is [rows, K] bf16, K-major (the activations). B is [groups, K, N] bf16 with
+// N contiguous (the weights exactly as given), which the tensor core reads as
+// an MN-major operand, so no weight is repacked.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile 128x64 and B chunks 64(K)x64(N) per stage
+//   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
+//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator, apply GeGLU or
+//               convert, store rows that belong to the tile
+// Shared memory: 4 stages x (16 KB A + 32 KB B), 128-byte swizzle.
+// TMEM: 2 accumulator buffers x 256 fp32 columns, so the epilogue of one tile
+// overlaps the main loop of the next.
+//
+// GATEUP tiles put 64-column chunks of the gate weights and the same columns
+// of the up weights side by side in shared memory, so ONE MMA of N = 2*wn
+// computes both projections of wn output columns (wn = 128, or 64 for the
+// last columns): TMEM columns [0, wn) hold x Bg, [wn, 2 wn) hold x Bu.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kAStageBytes = kBM * kBK * 2;   // 16 KB
+constexpr int kBChunkBytes = kBK * 64 * 2;    // 8 KB: 64 K-rows x 64 N-columns
+constexpr int kMaxBChunks = 4;
+constexpr int kBStageBytes = kMaxBChunks * kBChunkBytes;
+constexpr int kAccCols = 256;
+constexpr int kTmemCols = 512;
+constexpr int kGemmThreads = 192;
+constexpr int kGemmSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 /*align*/ + 256 /*barriers*/;
+
+// One 128-row work tile. pg = (problem << 16) | group.
+struct Tile {
+  int32_t pg;
+  int32_t row0;  // first A row
+  int32_t rows;  // rows of A that belong to this tile (1..128)
+  int32_t n0;    // first output column (per projection for GATEUP)
+};
+
+struct GemmProblem {
+  int K;        // reduction length, multiple of 64
+  int N;        // output columns, multiple of 64
+  int groups;   // number of B matrices (range check)
+  int a_rows;   // rows of A (range check)
+  void* out;    // [a_rows, ldo] bf16 or fp32
+  int ldo;
+  int out_f32;
+};
+
+struct GemmParams {
+  CUtensorMap tmA[2];   // [a_rows, K] bf16, box 64 x 128
+  CUtensorMap tmB0[2];  // [groups, K, N] bf16, box 64 x 64 x 1 (gate, or the only B)
+  CUtensorMap tmB1[2];  // [groups, K, N] bf16 (up; GATEUP only)
+  GemmProblem prob[2];
+  int nprob;
+  const Tile* tiles;
+  const int32_t* num_tiles;
+  uint32_t* err;
+};
+
+template <bool GATEUP>
+__device__ __forceinline__ int tile_cols(const GemmProblem& pr, int n0) {
+  const int cap = GATEUP ? 128 : 256;
+  const int rem = pr.N - n0;
+  return rem < cap ? rem : cap;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kStages * kAStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * (kAStageBytes + kBStageBytes));
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int p = 0; p < P.nprob; ++p) {
+      tma_prefetch_desc(&P.tmA[p]);
+      tma_prefetch_desc(&P.tmB0[p]);
+      if (GATEUP) tma_prefetch_desc(&P.tmB1[p]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_tiles = *P.num_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+        const Tile tile = P.tiles[ti];
+        const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+        if (p >= P.nprob) {
+          atomicOr(P.err, kErrBadTile);
+          *abort_flag = 1;
+          break;
+        }
+        const GemmProblem& pr = P.prob[p];
+        if (g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || tile.n0 < 0 || tile.n0 >= pr.N) {
+          atomicOr(P.err, kErrBadTile);
+          *abort_flag = 1;
+          break;
+        }
+        const int wn = tile_cols<GATEUP>(pr, tile.n0);
+        const int cpp = wn >> 6;  // 64-column chunks per projection
+        const int nch = GATEUP ? 2 * cpp : cpp;
+        const uint32_t bytes = kAStageBytes + nch * kBChunkBytes;
+        const int nkb = pr.K / kBK;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d(sA + s * kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row0);
+          for (int c = 0; c < nch; ++c) {
+            const bool up = GATEUP && c >= cpp;
+            const int col = tile.n0 + (up ? c - cpp : c) * 64;
+            tma_load_3d(sB + s * kBStageBytes + c * kBChunkBytes, up ? &P.tmB1[p] : &P.tmB0[p], &full[s], col,
+                        kb * kBK, g);
+          }
+          ++issued;
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA's memory goes away
+        int st = s;
+        uint32_t sp = ph;
+        const int pending = issued < kStages ? issued : kStages;
+        for (int i = 0; i < pending; ++i) {
+          if (--st < 0) {
+            st = kStages - 1;
+            sp ^= 1;
+          }
+          uint32_t dummy = 0;
+          mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      int s = 0, acc = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool any = false;
+      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+        const Tile tile = P.tiles[ti];
+        const int p = tile.pg >> 16;
+        if (p >= P.nprob) break;
+        const GemmProblem& pr = P.prob[p];
+        const int wn = tile_cols<GATEUP>(pr, tile.n0);
+        const int n_mma = GATEUP ? 2 * wn : wn;
+        const uint32_t idesc = idesc_bf16_m128(n_mma, 1);
+        const int nkb = pr.K / kBK;
+        if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag, P.err)) break;
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_addr = smem_u32(sA + s * kAStageBytes);
+          const uint32_t b_addr = smem_u32(sB + s * kBStageBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // A: K-major, rows of 128 B, 8-row groups 1024 B apart; +32 B per 16 K.
+            const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
+            // B: N-major; 8 K-rows form a 1024 B swizzle atom (SBO), 64-column
+            // chunks are 8 KB apart (LBO); +16 K-rows = +2048 B.
+            const uint64_t bd = sdesc_sw128(b_addr + k * 2048, kBChunkBytes, 1024);
+            umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          any = true;
+          umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);  // accumulator complete
+        if (++acc == 2) {
+          acc = 0;
+          acc_ph ^= 1;
+        }
+      }
+      if (any) {
+        // all MMAs of this CTA have finished before TMEM is released
+        umma_commit(drain);
+        uint32_t dummy = 0;
+        mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), P.err);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter..+31
+    const int r = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      const Tile tile = P.tiles[ti];
+      const int p = tile.pg >> 16;
+      if (p >= P.nprob) break;
+      const GemmProblem& pr = P.prob[p];
+      const int wn = tile_cols<GATEUP>(pr, tile.n0);
+      const bool ready = mbar_wait(&acc_full[acc], acc_ph, abort_flag, P.err);
+      __syncwarp();
+      if (!ready) break;
+      tc_fence_after_sync();
+      const uint32_t tbase = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+      const bool valid = r < tile.rows;
+      const size_t grow = static_cast<size_t>(tile.row0 + r);
+      if (GATEUP) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo + tile.n0;
+        for (int j = 0; j < wn; j += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld_32x32b_x32(tbase + j, g);
+          tmem_ld_32x32b_x32(tbase + wn + j, u);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float h0 = gelu_tanh(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+            const float h1 = gelu_tanh(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+            pk[i] = pack_bf16x2(h0, h1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(out + j);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      } else {
+        for (int j = 0; j < wn; j += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(tbase + j, a);
+          tmem_ld_wait();
+          if (valid) {
+            if (pr.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + grow * pr.ldo + tile.n0 + j);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                                     __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo +
+                                                    tile.n0 + j);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
+                                    pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
+                                    pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
+                                    pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])));
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_ph ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,645 @@
+// C ABI of the MoE feed-forward block (declared in include/moe_block.h):
+// host-side validation, workspace layout, TMA descriptors and the launch
+// sequence router -> top-k -> scan -> scatter -> gather -> gate|up GEMM ->
+// down GEMM -> combine, all on the caller's stream with no host sync.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "moe_block.h"
+#include "grouped_gemm.cuh"
+#include "permute.cuh"
+#include "router.cuh"
+
+namespace moe {
+
+__device__ uint32_t g_device_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kSmCountHint = 148;  // B200: sizes the router's split of the reduction
+constexpr size_t kAlign = 256;
+
+thread_local int t_launches = 0;
+
+struct Dims {
+  int T, k, D, E, F, S;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+  size_t total;
+  size_t partial, idx, w, chunk_cnt, cnt, off, row_of, token_of, tiles_gu, tiles_dn, counts;
+  size_t x_perm, h, y, hs, s;
+  int nsplit, nchunks, max_tiles_gu, max_tiles_dn;
+};
+
+int router_splits(const Dims& d) {
+  const int tiles = std::max(1, (d.T + kRouterTokens - 1) / kRouterTokens);
+  int ns = (2 * kSmCountHint + tiles - 1) / tiles;
+  ns = std::min(ns, 22);
+  ns = std::min(ns, d.D / kRouterKChunk);
+  return std::max(ns, 1);
+}
+
+Layout make_layout(const Dims& d) {
+  Layout L{};
+  const size_t T = d.T, k = d.k, E = d.E, R = T * k;
+  L.nsplit = router_splits(d);
+  L.nchunks = static_cast<int>((T + kTopkChunk - 1) / kTopkChunk);
+  const int mt_sh = static_cast<int>((T + kBM - 1) / kBM);
+  const long long mt_max = static_cast<long long>(R / kBM) + std::min<long long>(E, R) + 1;
+  L.max_tiles_gu = static_cast<int>(((d.S + 127) / 128) * mt_sh + mt_max * ((d.F + 127) / 128));
+  L.max_tiles_dn = static_cast<int>(((d.D + 255) / 256) * mt_sh + mt_max * ((d.D + 255) / 256));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, kAlign);
+    return at;
+  };
+  L.partial = take(static_cast<size_t>(L.nsplit) * T * E * 4);
+  L.idx = take(R * 4);
+  L.w = take(R * 4);
+  L.chunk_cnt = take(static_cast<size_t>(L.nchunks) * E * 4);
+  L.cnt = take(E * 4);
+  L.off = take((E + 1) * 4);
+  L.row_of = take(R * 4);
+  L.token_of = take(R * 4);
+  L.tiles_gu = take(static_cast<size_t>(L.max_tiles_gu) * sizeof(Tile));
+  L.tiles_dn = take(static_cast<size_t>(L.max_tiles_dn) * sizeof(Tile));
+  L.counts = take(sizeof(TileCounts));
+  L.x_perm = take(R * d.D * 2);
+  L.h = take(R * d.F * 2);
+  L.y = take(R * d.D * 2);
+  L.hs = take(T * d.S * 2);
+  L.s = take(T * d.D * 4);
+  L.total = o;
+  return L;
+}
+
+Dims dims_of(const moe_params* p) {
+  Dims d;
+  d.T = p->T;
+  d.k = p->top_k_experts;
+  d.D = p->embed_dim ? p->embed_dim : MOE_EMBED_DIM;
+  d.E = p->num_experts ? p->num_experts : MOE_NUM_EXPERTS;
+  d.F = p->expert_dim ? p->expert_dim : MOE_EXPERT_DIM;
+  d.S = p->hidden_dim ? p->hidden_dim : MOE_HIDDEN_DIM;
+  return d;
+}
+
+bool dims_ok(const Dims& d) {
+  if (d.T < 0) return false;
+  if (d.D <= 0 || d.F <= 0 || d.S <= 0 || d.D % 64 || d.F % 64 || d.S % 64) return false;
+  if (d.E < 8 || d.E > 128 || d.E % 8) return false;
+  if (d.k < 1 || d.k > d.E) return false;
+  if (static_cast<long long>(d.T) * d.k > (1LL << 30)) return false;
+  return true;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+
+// ---------------------------------------------------------- per-device state
+
+std::mutex g_mutex;
+struct DeviceState {
+  bool init = false;
+  bool arch_ok = false;
+  int sm_count = 0;
+  uint32_t* err = nullptr;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+};
+DeviceState g_dev[kMaxDevices];
+
+moe_status device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& s = g_dev[dev];
+  if (!s.init) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+    s.arch_ok = prop.major == 10 && prop.minor == 0;
+    s.sm_count = prop.multiProcessorCount;
+    if (s.arch_ok) {
+      if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), g_device_error) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kGemmSmemBytes) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kGemmSmemBytes) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    s.init = true;
+  }
+  if (!s.arch_ok) return MOE_ERR_ARCH;
+  *out = &s;
+  return MOE_OK;
+}
+
+// Library-owned workspace, grown on demand (one per device).
+moe_status library_workspace(DeviceState* s, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (s->ws_bytes < bytes) {
+    if (s->ws) {
+      cudaDeviceSynchronize();
+      cudaFree(s->ws);
+      s->ws = nullptr;
+      s->ws_bytes = 0;
+    }
+    if (cudaMalloc(&s->ws, bytes) != cudaSuccess) {
+      s->ws = nullptr;
+      return MOE_ERR_CUDA;
+    }
+    s->ws_bytes = bytes;
+  }
+  *out = s->ws;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [rows, cols] bf16 row-major; box = 64 columns x box_rows rows; 128-byte swizzle.
+bool map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [groups, K, N] bf16 with N contiguous; box = 64 (N) x 64 (K) x 1; 128-byte swizzle.
+bool map_3d(CUtensorMap* m, const void* base, uint64_t groups, uint64_t K, uint64_t N) {
+  const cuuint64_t dims[3] = {N, K, groups};
+  const cuuint64_t strides[2] = {N * 2, K * N * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Kernel ids of the per-kernel timing records.
+enum KernelId : int {
+  kKRouterLogits = 0,
+  kKRouterTopk,
+  kKChunkHistogram,
+  kKRouteScan,
+  kKRouteScatter,
+  kKGatherRows,
+  kKGemmGateUp,
+  kKGemmDown,
+  kKCombine,
+  kKTimeoutProbe,
+  kKCount
+};
+const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "chunk_histogram", "route_scan",
+                                           "route_scatter", "gather_rows", "grouped_gemm_gateup",
+                                           "grouped_gemm_down", "combine", "timeout_probe"};
+
+struct ProfRecord {
+  int id;
+  cudaEvent_t start, stop;
+};
+thread_local bool t_profiling = false;
+thread_local std::vector<ProfRecord> t_records;
+thread_local std::vector<cudaEvent_t> t_event_pool;
+
+cudaEvent_t pooled_event() {
+  if (!t_event_pool.empty()) {
+    cudaEvent_t e = t_event_pool.back();
+    t_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets one kernel launch with timing events when profiling is on.
+struct LaunchScope {
+  cudaStream_t st;
+  int id;
+  cudaEvent_t a = nullptr;
+  LaunchScope(int id_, cudaStream_t st_) : st(st_), id(id_) {
+    if (t_profiling) {
+      a = pooled_event();
+      cudaEventRecord(a, st);
+    }
+  }
+  moe_status done() {
+    ++t_launches;
+    if (t_profiling && a) {
+      cudaEvent_t b = pooled_event();
+      cudaEventRecord(b, st);
+      t_records.push_back(ProfRecord{id, a, b});
+    }
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+};
+
+#define MOE_TRY(expr)                   \
+  do {                                  \
+    const moe_status st_ = (expr);      \
+    if (st_ != MOE_OK) return st_;      \
+  } while (0)
+
+// ------------------------------------------------------------- validation
+
+moe_status check_block_args(const moe_params* p, Dims* d) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  *d = dims_of(p);
+  if (!dims_ok(*d)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  const void* req[] = {p->x, p->w_router, p->wg, p->wu, p->wd, p->sg, p->su, p->sd, p->out};
+  for (const void* q : req)
+    if (!q) return MOE_ERR_INVALID_ARG;
+  for (const void* q : req)
+    if (!aligned16(q)) return MOE_ERR_ALIGNMENT;
+  if (p->out_f32 && !aligned16(p->out_f32)) return MOE_ERR_ALIGNMENT;
+  const void* opt4[] = {p->router_bias, p->idx_out, p->w_out, p->cnt_out};
+  for (const void* q : opt4)
+    if (q && !aligned4(q)) return MOE_ERR_ALIGNMENT;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(p->x), ob = reinterpret_cast<uintptr_t>(p->out);
+  const uintptr_t bytes = static_cast<uintptr_t>(d->T) * d->D * 2;
+  if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status resolve_workspace(const moe_params* p, DeviceState* s, const Layout& L, uint8_t** ws) {
+  if (p->workspace) {
+    if ((reinterpret_cast<uintptr_t>(p->workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGNMENT;
+    if (p->workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    *ws = static_cast<uint8_t*>(p->workspace);
+    return MOE_OK;
+  }
+  void* w = nullptr;
+  MOE_TRY(library_workspace(s, L.total, &w));
+  *ws = static_cast<uint8_t*>(w);
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- stages
+
+moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void* x, const void* wr,
+                         const float* bias, int32_t* idx, float* w, cudaStream_t st) {
+  float* partial = reinterpret_cast<float*>(ws + L.partial);
+  const dim3 g1((d.T + kRouterTokens - 1) / kRouterTokens, L.nsplit);
+  {
+  LaunchScope ls_(kKRouterLogits, st);
+  router_logits_kernel<<<g1, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                      static_cast<const __nv_bfloat16*>(wr), partial, d.T, d.D, d.E,
+                                                      L.nsplit);
+  MOE_TRY(ls_.done());
+  }
+  {
+  LaunchScope ls_(kKRouterTopk, st);
+  router_topk_kernel<<<L.nchunks, kTopkThreads, 0, st>>>(partial, bias, d.T, d.E, L.nsplit, d.k, idx, w,
+                                                         reinterpret_cast<int32_t*>(ws + L.chunk_cnt));
+  return ls_.done();
+  }
+}
+
+moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const int32_t* idx, int32_t* cnt,
+                           int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st) {
+  int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
+  {
+  LaunchScope ls_(kKRouteScan, st);
+  route_scan_kernel<<<1, 128, 0, st>>>(chunk, L.nchunks, d.T, d.E, d.F, d.S, d.D, cnt, off,
+                                       reinterpret_cast<Tile*>(ws + L.tiles_gu),
+                                       reinterpret_cast<Tile*>(ws + L.tiles_dn),
+                                       reinterpret_cast<TileCounts*>(ws + L.counts));
+  MOE_TRY(ls_.done());
+  }
+  {
+  LaunchScope ls_(kKRouteScatter, st);
+  route_scatter_kernel<<<L.nchunks, 128, 0, st>>>(idx, chunk, d.T, d.k, d.E, row_of, token_of);
+  return ls_.done();
+  }
+}
+
+moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, uint8_t* ws, DeviceState* s,
+                         cudaStream_t st) {
+  const size_t R = static_cast<size_t>(d.T) * d.k;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  int32_t* off = reinterpret_cast<int32_t*>(ws + L.off);
+  int32_t* row_of = reinterpret_cast<int32_t*>(ws + L.row_of);
+  int32_t* token_of = reinterpret_cast<int32_t*>(ws + L.token_of);
+  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+  __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(ws + L.hs);
+  float* sbuf = reinterpret_cast<float*>(ws + L.s);
+  const TileCounts* counts = reinterpret_cast<const TileCounts*>(ws + L.counts);
+
+  MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
+  MOE_TRY(enqueue_permute(d, L, ws, idx, cnt, off, row_of, token_of, st));
+
+  const int gather_blocks = static_cast<int>(std::min<size_t>((R + 7) / 8, static_cast<size_t>(s->sm_count) * 16));
+  {
+  LaunchScope ls_(kKGatherRows, st);
+  gather_rows_kernel<<<gather_blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(p->x), token_of,
+                                                    static_cast<int>(R), d.D, x_perm);
+  MOE_TRY(ls_.done());
+  }
+
+  // gate|up: experts (problem 0) and shared MLP (problem 1)
+  GemmParams gu;
+  std::memset(&gu, 0, sizeof(gu));
+  bool ok = map_2d(&gu.tmA[0], x_perm, R, d.D, kBM) && map_3d(&gu.tmB0[0], p->wg, d.E, d.D, d.F) &&
+            map_3d(&gu.tmB1[0], p->wu, d.E, d.D, d.F) && map_2d(&gu.tmA[1], p->x, d.T, d.D, kBM) &&
+            map_3d(&gu.tmB0[1], p->sg, 1, d.D, d.S) && map_3d(&gu.tmB1[1], p->su, 1, d.D, d.S);
+  if (!ok) return MOE_ERR_CUDA;
+  gu.prob[0] = GemmProblem{d.D, d.F, d.E, static_cast<int>(R), h, d.F, 0};
+  gu.prob[1] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
+  gu.nprob = 2;
+  gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
+  gu.num_tiles = &counts->gateup;
+  gu.err = s->err;
+  const int grid_gu = std::min(s->sm_count, L.max_tiles_gu);
+  {
+  LaunchScope ls_(kKGemmGateUp, st);
+  grouped_gemm_kernel<true><<<grid_gu, kGemmThreads, kGemmSmemBytes, st>>>(gu);
+  MOE_TRY(ls_.done());
+  }
+
+  // down: experts -> y (bf16), shared -> s (fp32)
+  GemmParams dn;
+  std::memset(&dn, 0, sizeof(dn));
+  ok = map_2d(&dn.tmA[0], h, R, d.F, kBM) && map_3d(&dn.tmB0[0], p->wd, d.E, d.F, d.D) &&
+       map_2d(&dn.tmA[1], hs, d.T, d.S, kBM) && map_3d(&dn.tmB0[1], p->sd, 1, d.S, d.D);
+  if (!ok) return MOE_ERR_CUDA;
+  dn.tmB1[0] = dn.tmB0[0];
+  dn.tmB1[1] = dn.tmB0[1];
+  dn.prob[0] = GemmProblem{d.F, d.D, d.E, static_cast<int>(R), y, d.D, 0};
+  dn.prob[1] = GemmProblem{d.S, d.D, 1, d.T, sbuf, d.D, 1};
+  dn.nprob = 2;
+  dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
+  dn.num_tiles = &counts->down;
+  dn.err = s->err;
+  const int grid_dn = std::min(s->sm_count, L.max_tiles_dn);
+  {
+  LaunchScope ls_(kKGemmDown, st);
+  grouped_gemm_kernel<false><<<grid_dn, kGemmThreads, kGemmSmemBytes, st>>>(dn);
+  MOE_TRY(ls_.done());
+  }
+
+  {
+  LaunchScope ls_(kKCombine, st);
+  combine_kernel<<<d.T, 128, 0, st>>>(sbuf, y, row_of, w, d.T, d.k, d.D, static_cast<__nv_bfloat16*>(p->out),
+                                      p->out_f32);
+  MOE_TRY(ls_.done());
+  }
+
+  if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->w_out && cudaMemcpyAsync(p->w_out, w, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->cnt_out && cudaMemcpyAsync(p->cnt_out, cnt, d.E * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes_ex(const moe_params* p) {
+  if (!p) return 0;
+  const Dims d = dims_of(p);
+  if (!dims_ok(d)) return 0;
+  return make_layout(d).total;
+}
+
+size_t moe_workspace_bytes(int T, int top_k) {
+  moe_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.T = T;
+  p.top_k_experts = top_k;
+  return moe_workspace_bytes_ex(&p);
+}
+
+moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out) {
+  if (!p || !out) return MOE_ERR_INVALID_ARG;
+  const Dims d = dims_of(p);
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(d);
+  out->total_bytes = L.total;
+  out->x_perm = L.x_perm;
+  out->h = L.h;
+  out->y = L.y;
+  out->hs = L.hs;
+  out->s = L.s;
+  out->idx = L.idx;
+  out->w = L.w;
+  out->cnt = L.cnt;
+  out->off = L.off;
+  out->row_of = L.row_of;
+  out->token_of = L.token_of;
+  return MOE_OK;
+}
+
+moe_status moe_block_forward_ex(const moe_params* p, void* stream) {
+  t_launches = 0;
+  Dims d;
+  MOE_TRY(check_block_args(p, &d));
+  if (d.T == 0) return MOE_OK;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  const Layout L = make_layout(d);
+  uint8_t* ws = nullptr;
+  MOE_TRY(resolve_workspace(p, s, L, &ws));
+  return enqueue_block(p, d, L, ws, s, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_block_forward(const void* x, const void* w_router, const void* wg, const void* wu, const void* wd,
+                             const void* sg, const void* su, const void* sd, int T, void* out, void* stream) {
+  moe_params p;
+  std::memset(&p, 0, sizeof(p));
+  p.T = T;
+  p.top_k_experts = MOE_TOP_K;
+  p.x = x;
+  p.w_router = w_router;
+  p.wg = wg;
+  p.wu = wu;
+  p.wd = wd;
+  p.sg = sg;
+  p.su = su;
+  p.sd = sd;
+  p.out = out;
+  return moe_block_forward_ex(&p, stream);
+}
+
+moe_status moe_route(const moe_params* p, int32_t* idx, float* w, void* stream) {
+  t_launches = 0;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  const Dims d = dims_of(p);
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  if (d.T == 0) return MOE_OK;
+  if (!p->x || !p->w_router || !idx || !w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned4(idx) || !aligned4(w)) return MOE_ERR_ALIGNMENT;
+  if (p->router_bias && !aligned4(p->router_bias)) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  const Layout L = make_layout(d);
+  uint8_t* ws = nullptr;
+  MOE_TRY(resolve_workspace(p, s, L, &ws));
+  return enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_permute(const moe_params* p, const int32_t* idx, int32_t* cnt, int32_t* off, int32_t* row_of,
+                       int32_t* token_of, void* stream) {
+  t_launches = 0;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  const Dims d = dims_of(p);
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  if (d.T == 0) return MOE_OK;
+  if (!idx || !cnt || !off || !row_of || !token_of) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {idx, cnt, off, row_of, token_of};
+  for (const void* q : ptrs)
+    if (!aligned4(q)) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  const Layout L = make_layout(d);
+  uint8_t* ws = nullptr;
+  MOE_TRY(resolve_workspace(p, s, L, &ws));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+  LaunchScope ls_(kKChunkHistogram, st);
+  chunk_histogram_kernel<<<L.nchunks, 128, 0, st>>>(idx, d.T, d.k, d.E, reinterpret_cast<int32_t*>(ws + L.chunk_cnt),
+                                                     s->err);
+  MOE_TRY(ls_.done());
+  }
+  return enqueue_permute(d, L, ws, idx, cnt, off, row_of, token_of, st);
+}
+
+moe_status moe_get_device_status(void* stream) {
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, s->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word) {
+    if (cudaMemset(s->err, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
+    return (word & kErrWaitTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_debug_timeout_probe(int timeout_us, void* stream) {
+  t_launches = 0;
+  if (timeout_us <= 0 || timeout_us > 10000000) return MOE_ERR_INVALID_ARG;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  {
+  LaunchScope ls_(kKTimeoutProbe, static_cast<cudaStream_t>(stream));
+  timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      s->err, static_cast<unsigned long long>(timeout_us) * 1000ull);
+  return ls_.done();
+  }
+}
+
+const char* moe_status_string(moe_status st) {
+  switch (st) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_ARCH: return "MOE_ERR_ARCH";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int moe_last_launch_count(void) { return t_launches; }
+
+moe_status moe_block_forward_hostio(const moe_params* p, const void* x_host, void* out_host, void* stream) {
+  t_launches = 0;
+  Dims d;
+  MOE_TRY(check_block_args(p, &d));
+  if (d.T == 0) return MOE_OK;
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(d.T) * d.D * 2;
+  if (cudaMemcpyAsync(const_cast<void*>(p->x), x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  const Layout L = make_layout(d);
+  uint8_t* ws = nullptr;
+  MOE_TRY(resolve_workspace(p, s, L, &ws));
+  MOE_TRY(enqueue_block(p, d, L, ws, s, st));
+  if (cudaMemcpyAsync(out_host, p->out, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_profile_begin(void) {
+  for (const ProfRecord& r : t_records) {
+    t_event_pool.push_back(r.start);
+    t_event_pool.push_back(r.stop);
+  }
+  t_records.clear();
+  t_profiling = true;
+  return MOE_OK;
+}
+
+int moe_profile_end(float* total_ms, int* launches, int n) {
+  t_profiling = false;
+  for (int i = 0; i < n; ++i) {
+    if (total_ms) total_ms[i] = 0.f;
+    if (launches) launches[i] = 0;
+  }
+  for (const ProfRecord& r : t_records) {
+    float ms = 0.f;
+    cudaEventSynchronize(r.stop);
+    cudaEventElapsedTime(&ms, r.start, r.stop);
+    if (r.id < n) {
+      if (total_ms) total_ms[r.id] += ms;
+      if (launches) launches[r.id] += 1;
+    }
+    t_event_pool.push_back(r.start);
+    t_event_pool.push_back(r.stop);
+  }
+  t_records.clear();
+  return kKCount;
+}
+
+const char* moe_kernel_name(int id) { return (id >= 0 && id < kKCount) ? kKernelNames[id] : nullptr; }
+
+}  // extern "C"

@@ -7,11 +7,11 @@ CUDA path and the CPU oracle can take their inputs from it.
 Recipe (no trained checkpoint is available, so weights are random-init of the
 published architecture):
 
-* weights: one ``numpy.random.default_rng(seed)`` stream, drawn in the order
+* weights: one seeded ``torch.Generator`` (CPU) stream, drawn in the order
   router, expert gate, expert up, expert down, shared gate, shared up, shared
-  down, each ``float32 N(0, 1) * 0.02`` (the checkpoint's
-  ``initializer_range`` 0.02), rounded to bf16 with round-to-nearest-even;
-* activations ``x``: ``default_rng(1)`` ``N(0, 1)`` rounded to bf16;
+  down, each float32 ``N(0, 0.02^2)`` (the checkpoint's ``initializer_range``
+  0.02), rounded to bf16 with round-to-nearest-even;
+* activations ``x``: seed 1, float32 ``N(0, 1)`` rounded to bf16;
 * the skewed-routing benchmark adds a per-expert router bias
   ``2.0 * ln(p_r)`` with ``p_r`` the Zipf(s=1.1) probability of rank
   ``r = e + 1`` over the experts.
@@ -57,11 +57,17 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def _normal_bf16(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
-    a = rng.standard_normal(size=shape, dtype=np.float32)
-    if scale != 1.0:
-        a *= np.float32(scale)
-    return f32_to_bf16_bits(a)
+def _normal_bf16(gen, shape, std: float) -> np.ndarray:
+    import torch
+
+    a = torch.empty(tuple(shape), dtype=torch.float32).normal_(0.0, std, generator=gen)
+    return a.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _generator(seed: int):
+    import torch
+
+    return torch.Generator().manual_seed(seed)
 
 
 @dataclasses.dataclass
@@ -83,7 +89,7 @@ class BlockWeights:
 
 def make_weights(dims: Dims = GEMMA4_26B_A4B, seed: int = 0, std: float = INIT_STD) -> BlockWeights:
     d, e, f, s = dims.embed_dim, dims.num_experts, dims.expert_dim, dims.hidden_dim
-    rng = np.random.default_rng(seed)
+    rng = _generator(seed)
     return BlockWeights(
         w_router=_normal_bf16(rng, (d, e), std),
         wg=_normal_bf16(rng, (e, d, f), std),
@@ -96,7 +102,7 @@ def make_weights(dims: Dims = GEMMA4_26B_A4B, seed: int = 0, std: float = INIT_S
 
 
 def make_x(tokens: int, embed_dim: int = EMBED_DIM, seed: int = 1) -> np.ndarray:
-    return _normal_bf16(np.random.default_rng(seed), (tokens, embed_dim), 1.0)
+    return _normal_bf16(_generator(seed), (tokens, embed_dim), 1.0)
 
 
 def zipf_router_bias(num_experts: int = NUM_EXPERTS, s: float = 1.1, amplitude: float = 2.0) -> np.ndarray:

@@ -1,0 +1,139 @@
+"""Shared helpers of the GPU parity tests: run the library, compare with the oracle."""
+
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_transformer_b200 import binding as B
+from mixture_experts_transformer_b200 import block, build, inputs
+from oracle import moe_oracle as mo
+
+# Output tolerance at the Gemma-4-26B-A4B shapes: max |err| <= 1e-2 * RMS(out)
+# on the fp32 pre-rounding output; routing compared exactly wherever the k-th /
+# (k+1)-th logit gap of the oracle exceeds 1e-4.
+OUT_TOL = 1e-2
+# At reduced test shapes the routed branch carries a larger share of the output
+# than in the real block (fewer, narrower experts), and the one deliberate
+# precision loss of the path - the bf16 storage of the GeGLU rows h and of the
+# expert outputs y, each rounded to nearest even (relative error <= 2^-8) - can
+# approach 1e-2 * RMS by itself. There the tolerance is derived from that
+# arithmetic: the test evaluates the oracle's formula with h and y rounded to
+# bf16 (float64 otherwise) to measure the rounding's own cost e_bf16, and allows
+# 1.25 * e_bf16 plus 2e-3 * RMS for fp32 accumulation and the tanh
+# approximation, or 1e-2 * RMS, whichever is larger.
+BF16_SLACK = 1.25
+ACC_SLACK = 2e-3
+GAP = 1e-4
+W_TOL = 2e-6
+
+SMALL = inputs.Dims(embed_dim=256, num_experts=16, expert_dim=192, hidden_dim=320)
+
+
+def require_gpu():
+    assert torch.cuda.is_available(), "the -m gpu tests need a CUDA device"
+    build.build()
+    B.lib()
+
+
+@functools.lru_cache(maxsize=4)
+def weights(dims: inputs.Dims = inputs.GEMMA4_26B_A4B, seed: int = 0, std: float = inputs.INIT_STD):
+    return inputs.make_weights(dims, seed=seed, std=std)
+
+
+@functools.lru_cache(maxsize=4)
+def device_weights(dims: inputs.Dims = inputs.GEMMA4_26B_A4B, seed: int = 0, std: float = inputs.INIT_STD):
+    return block.upload(weights(dims, seed, std))
+
+
+def w_args(w: inputs.BlockWeights):
+    return (w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def bf16_to_f32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy()
+
+
+def run_block(dw, x_bits, top_k=8, bias=None, workspace=None):
+    x = block.bf16_tensor(x_bits)
+    b = None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).cuda()
+    res = block.forward(dw, x, top_k=top_k, router_bias=b, debug=True, workspace=workspace)
+    st = B.moe_get_device_status()
+    assert st == B.MOE_OK, B.moe_status_string(st)
+    return res
+
+
+def rne_bf16(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def check_routing(ref_logits, ref_idx, ref_w, idx, w, k):
+    """Expert sets exact where the k/k+1 gap is clear; slot order where adjacent gaps are clear."""
+    gap = mo.top_k_gap(ref_logits, k)
+    clear = gap > GAP
+    assert clear.mean() > 0.9, clear.mean()
+    for t in np.flatnonzero(clear):
+        assert sorted(idx[t]) == sorted(ref_idx[t]), (t, idx[t], ref_idx[t])
+    s = -np.sort(-ref_logits, axis=1)[:, :k]
+    order_clear = np.all(-np.diff(s, axis=1) > GAP, axis=1) & clear
+    np.testing.assert_array_equal(idx[order_clear], ref_idx[order_clear])
+    np.testing.assert_allclose(w[order_clear], ref_w[order_clear], rtol=0, atol=W_TOL)
+    # every token: k distinct experts, weights sum to one and do not increase
+    assert all(len(set(r)) == k for r in idx)
+    np.testing.assert_allclose(w.sum(1), 1.0, atol=1e-5)
+    assert np.all(np.diff(w, axis=1) <= 1e-7)
+    return clear
+
+
+def _rne_bf16_f64(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def bf16_storage_cost(xs, w_host, idx, wts):
+    """max |out(h, y rounded to bf16) - out(exact)| for the given routing (CPU, float64)."""
+    x = mo.f64(xs)
+    exact = np.zeros((x.shape[0], x.shape[1]))
+    rounded = np.zeros_like(exact)
+    for e in np.unique(idx):
+        tok, slot = np.nonzero(idx == e)
+        h = mo.geglu_hidden(x[tok], w_host.wg[e], w_host.wu[e])
+        wd = mo.f64(w_host.wd[e])
+        wk = wts[tok, slot][:, None]
+        exact[tok] += wk * (h @ wd)
+        rounded[tok] += wk * _rne_bf16_f64(_rne_bf16_f64(h) @ wd)
+    return np.abs(rounded - exact).max()
+
+
+def check_block_output(w_host, x_bits, res, k, bias=None, tokens=None, derived_tol=False):
+    """Oracle on (a subset of) tokens: routing per check_routing, output within
+    tolerance given the GPU's own routing, and out == RNE(out_f32) exactly.
+    derived_tol=False: the 1e-2 * RMS bound (Gemma shapes); True: the bound
+    derived from the bf16 storage of h and y (reduced shapes)."""
+    tok = np.arange(x_bits.shape[0]) if tokens is None else np.asarray(tokens)
+    xs = x_bits[tok]
+    idx = to_np(res.idx)[tok]
+    wts = to_np(res.w)[tok]
+    ref = mo.moe_block(xs, *w_args(w_host), top_k=k, bias=bias)
+    check_routing(ref["logits"], ref["idx"], ref["w"], idx, wts, k)
+    ref_g = mo.moe_block(xs, *w_args(w_host), routing=(idx, wts))
+    out32 = to_np(res.out_f32)[tok].astype(np.float64)
+    rms = np.sqrt(np.mean(ref_g["out"] ** 2))
+    err = np.abs(out32 - ref_g["out"]).max()
+    bound = OUT_TOL * rms
+    if derived_tol:
+        bound = max(bound, BF16_SLACK * bf16_storage_cost(xs, w_host, idx, wts) + ACC_SLACK * rms)
+    assert err <= bound, (err, rms, err / rms, bound / rms)
+    np.testing.assert_array_equal(bf16_to_f32(res.out)[tok], rne_bf16(to_np(res.out_f32)[tok]))
+    return err / rms
+
+
+def skip_unless(cond, why):
+    if not cond:
+        pytest.skip(why)

@@ -1,0 +1,86 @@
+"""The C-ABI library loads, exports every declared entry point and validates
+arguments on the host (no GPU needed: every case here returns before any
+CUDA call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from mixture_experts_transformer_b200 import binding as B
+from mixture_experts_transformer_b200 import build as mbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mbuild.build()
+    return B.lib()
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if not f.endswith(".h"):
+            continue
+        src = open(os.path.join(inc, f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(moe_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(B.EXPORTS), set(names) - set(B.EXPORTS)
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert B.moe_status_string(code).startswith("MOE_")
+
+
+def test_workspace_sizes(lib):
+    assert B.moe_workspace_bytes(0) > 0
+    small = B.moe_workspace_bytes(8)
+    big = B.moe_workspace_bytes(4096)
+    assert big > small > 0
+    # the routed intermediates dominate: x_perm, y (bf16 [8T, 2816]) and h
+    assert big >= 4096 * 8 * (2816 * 2 * 2 + 704 * 2)
+    p = B.make_params(64)
+    lay = B.moe_workspace_layout(p)
+    offs = [lay.x_perm, lay.h, lay.y, lay.hs, lay.s, lay.idx, lay.w, lay.cnt, lay.off, lay.row_of, lay.token_of]
+    assert all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == len(offs)
+    assert lay.total_bytes == B.moe_workspace_bytes(64)
+    assert B.moe_workspace_bytes(64, 0) == 0  # top_k 0 is invalid
+
+
+def _params(**kw):
+    base = dict(x=16, w_router=16, wg=16, wu=16, wd=16, sg=16, su=16, sd=16, out=1 << 40)
+    base.update(kw)
+    return B.make_params(kw.pop("T", 4), **{k: v for k, v in base.items() if k != "T"})
+
+
+def test_host_validation(lib):
+    f = lambda p: lib.moe_block_forward_ex(ctypes.byref(p), None)  # noqa: E731
+    assert f(_params(T=0)) == B.MOE_OK  # empty batch: no-op
+    assert f(_params(T=-1)) == B.MOE_ERR_INVALID_ARG
+    assert f(_params(x=0)) == B.MOE_ERR_INVALID_ARG  # null x
+    assert f(_params(x=18)) == B.MOE_ERR_ALIGNMENT
+    assert f(_params(out=16)) == B.MOE_ERR_INVALID_ARG  # out aliases x
+    p = _params()
+    p.top_k_experts = 129
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params()
+    p.expert_dim = 700  # not a multiple of 64
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params()
+    p.num_experts = 256  # more than one warp's 4 experts per lane
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_block_forward_ex(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_debug_timeout_probe(0, None) == B.MOE_ERR_INVALID_ARG
