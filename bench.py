@@ -225,7 +225,7 @@ def algorithmic(kernel: str, T: int, touched: int, cnt: np.ndarray):
     elif kernel == "grouped_gemm_down":
         byts = touched * F * D * 2 + S * D * 2 + R * F * 2 + T * S * 2 + R * D * 2 + T * D * 4
         flops = 2 * D * (R * F + T * S)
-    elif kernel == "gather_rows":
+    elif kernel == "route_scatter":
         byts = T * D * 2 + R * D * 2
         flops = 0
     elif kernel == "combine":

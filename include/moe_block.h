@@ -163,7 +163,9 @@ moe_status moe_route(const moe_params* p, int32_t* idx, float* w, void* stream);
 
 /*
  * Expert-major permutation of the (token, slot) assignments in idx
- * [T, top_k] (values in [0, num_experts)): cnt [num_experts] tokens per
+ * [T, top_k] (values in [0, num_experts), distinct within a row, as the
+ * router produces them; out-of-range values are skipped and reported by
+ * moe_get_device_status): cnt [num_experts] tokens per
  * expert, off [num_experts + 1] exclusive scan of cnt, row_of [T, top_k]
  * routed row of each assignment, token_of [T * top_k] token of each row. Rows
  * of expert e are off[e] .. off[e+1]-1 in ascending token order. Integer

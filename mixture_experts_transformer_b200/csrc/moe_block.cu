@@ -36,7 +36,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
   size_t total;
-  size_t partial, idx, w, chunk_cnt, cnt, off, row_of, token_of, tiles_gu, tiles_dn, counts;
+  size_t partial, idx, w, masks, base, cnt, off, row_of, token_of, tiles_gu, tiles_dn, counts;
   size_t x_perm, h, y, hs, s;
   int nsplit, nchunks, max_tiles_gu, max_tiles_dn;
 };
@@ -53,7 +53,7 @@ Layout make_layout(const Dims& d) {
   Layout L{};
   const size_t T = d.T, k = d.k, E = d.E, R = T * k;
   L.nsplit = router_splits(d);
-  L.nchunks = static_cast<int>((T + kTopkChunk - 1) / kTopkChunk);
+  L.nchunks = static_cast<int>((T + kMaskTokens - 1) / kMaskTokens);
   const int mt_sh = static_cast<int>((T + kBM - 1) / kBM);
   const long long mt_max = static_cast<long long>(R / kBM) + std::min<long long>(E, R) + 1;
   L.max_tiles_gu = static_cast<int>(((d.S + 127) / 128) * mt_sh + mt_max * ((d.F + 127) / 128));
@@ -67,7 +67,8 @@ Layout make_layout(const Dims& d) {
   L.partial = take(static_cast<size_t>(L.nsplit) * T * E * 4);
   L.idx = take(R * 4);
   L.w = take(R * 4);
-  L.chunk_cnt = take(static_cast<size_t>(L.nchunks) * E * 4);
+  L.masks = take(static_cast<size_t>(L.nchunks) * E * 4);
+  L.base = take(static_cast<size_t>(L.nchunks) * E * 4);
   L.cnt = take(E * 4);
   L.off = take((E + 1) * 4);
   L.row_of = take(R * 4);
@@ -211,18 +212,17 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t groups, uint64_t K, uint6
 enum KernelId : int {
   kKRouterLogits = 0,
   kKRouterTopk,
-  kKChunkHistogram,
+  kKBuildMasks,
   kKRouteScan,
   kKRouteScatter,
-  kKGatherRows,
   kKGemmGateUp,
   kKGemmDown,
   kKCombine,
   kKTimeoutProbe,
   kKCount
 };
-const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "chunk_histogram", "route_scan",
-                                           "route_scatter", "gather_rows", "grouped_gemm_gateup",
+const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "build_masks", "route_scan",
+                                           "route_scatter", "grouped_gemm_gateup",
                                            "grouped_gemm_down", "combine", "timeout_probe"};
 
 struct ProfRecord {
@@ -312,38 +312,41 @@ moe_status resolve_workspace(const moe_params* p, DeviceState* s, const Layout& 
 moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void* x, const void* wr,
                          const float* bias, int32_t* idx, float* w, cudaStream_t st) {
   float* partial = reinterpret_cast<float*>(ws + L.partial);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(ws + L.masks);
   const dim3 g1((d.T + kRouterTokens - 1) / kRouterTokens, L.nsplit);
   {
-  LaunchScope ls_(kKRouterLogits, st);
-  router_logits_kernel<<<g1, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
-                                                      static_cast<const __nv_bfloat16*>(wr), partial, d.T, d.D, d.E,
-                                                      L.nsplit);
-  MOE_TRY(ls_.done());
+    LaunchScope ls_(kKRouterLogits, st);
+    router_logits_kernel<<<g1, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                        static_cast<const __nv_bfloat16*>(wr), partial, masks, d.T,
+                                                        d.D, d.E, L.nsplit);
+    MOE_TRY(ls_.done());
   }
-  {
   LaunchScope ls_(kKRouterTopk, st);
-  router_topk_kernel<<<L.nchunks, kTopkThreads, 0, st>>>(partial, bias, d.T, d.E, L.nsplit, d.k, idx, w,
-                                                         reinterpret_cast<int32_t*>(ws + L.chunk_cnt));
+  router_topk_kernel<<<(d.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(partial, bias, d.T, d.E,
+                                                                                     L.nsplit, d.k, idx, w, masks);
   return ls_.done();
-  }
 }
 
-moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const int32_t* idx, int32_t* cnt,
-                           int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st) {
-  int32_t* chunk = reinterpret_cast<int32_t*>(ws + L.chunk_cnt);
+// Scan of the bitmasks, then the scatter (and, with x, the gather into x_perm).
+moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const int32_t* idx, const void* x,
+                           int32_t* cnt, int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st) {
+  const uint32_t* masks = reinterpret_cast<const uint32_t*>(ws + L.masks);
+  int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   {
-  LaunchScope ls_(kKRouteScan, st);
-  route_scan_kernel<<<1, 128, 0, st>>>(chunk, L.nchunks, d.T, d.E, d.F, d.S, d.D, cnt, off,
-                                       reinterpret_cast<Tile*>(ws + L.tiles_gu),
-                                       reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                       reinterpret_cast<TileCounts*>(ws + L.counts));
-  MOE_TRY(ls_.done());
+    LaunchScope ls_(kKRouteScan, st);
+    route_scan_kernel<<<1, kScanThreads, 0, st>>>(masks, L.nchunks, d.T, d.E, d.F, d.S, d.D, base, cnt, off,
+                                                  reinterpret_cast<Tile*>(ws + L.tiles_gu),
+                                                  reinterpret_cast<Tile*>(ws + L.tiles_dn),
+                                                  reinterpret_cast<TileCounts*>(ws + L.counts));
+    MOE_TRY(ls_.done());
   }
-  {
+  const long long R = static_cast<long long>(d.T) * d.k;
+  const int blocks = static_cast<int>(std::min<long long>((R + 7) / 8, 148LL * 64));
   LaunchScope ls_(kKRouteScatter, st);
-  route_scatter_kernel<<<L.nchunks, 128, 0, st>>>(idx, chunk, d.T, d.k, d.E, row_of, token_of);
+  route_scatter_kernel<<<blocks, 256, 0, st>>>(idx, masks, base, d.T, d.k, d.E, d.D,
+                                               static_cast<const __nv_bfloat16*>(x), row_of, token_of,
+                                               reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm));
   return ls_.done();
-  }
 }
 
 moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, uint8_t* ws, DeviceState* s,
@@ -363,15 +366,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   const TileCounts* counts = reinterpret_cast<const TileCounts*>(ws + L.counts);
 
   MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
-  MOE_TRY(enqueue_permute(d, L, ws, idx, cnt, off, row_of, token_of, st));
-
-  const int gather_blocks = static_cast<int>(std::min<size_t>((R + 7) / 8, static_cast<size_t>(s->sm_count) * 16));
-  {
-  LaunchScope ls_(kKGatherRows, st);
-  gather_rows_kernel<<<gather_blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(p->x), token_of,
-                                                    static_cast<int>(R), d.D, x_perm);
-  MOE_TRY(ls_.done());
-  }
+  MOE_TRY(enqueue_permute(d, L, ws, idx, p->x, cnt, off, row_of, token_of, st));
 
   // gate|up: experts (problem 0) and shared MLP (problem 1)
   GemmParams gu;
@@ -416,8 +411,9 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
 
   {
   LaunchScope ls_(kKCombine, st);
-  combine_kernel<<<d.T, 128, 0, st>>>(sbuf, y, row_of, w, d.T, d.k, d.D, static_cast<__nv_bfloat16*>(p->out),
-                                      p->out_f32);
+  const int dsplit = std::max(1, std::min(4, (2 * s->sm_count) / std::max(1, d.T)));
+  combine_kernel<<<dim3(d.T, dsplit), 128, 0, st>>>(sbuf, y, row_of, w, d.T, d.k, d.D,
+                                                    static_cast<__nv_bfloat16*>(p->out), p->out_f32);
   MOE_TRY(ls_.done());
   }
 
@@ -538,13 +534,16 @@ moe_status moe_permute(const moe_params* p, const int32_t* idx, int32_t* cnt, in
   uint8_t* ws = nullptr;
   MOE_TRY(resolve_workspace(p, s, L, &ws));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t mask_bytes = static_cast<size_t>(L.nchunks) * d.E * 4;
+  if (cudaMemsetAsync(ws + L.masks, 0, mask_bytes, st) != cudaSuccess) return MOE_ERR_CUDA;
   {
-  LaunchScope ls_(kKChunkHistogram, st);
-  chunk_histogram_kernel<<<L.nchunks, 128, 0, st>>>(idx, d.T, d.k, d.E, reinterpret_cast<int32_t*>(ws + L.chunk_cnt),
-                                                     s->err);
-  MOE_TRY(ls_.done());
+    LaunchScope ls_(kKBuildMasks, st);
+    const long long R = static_cast<long long>(d.T) * d.k;
+    const int blocks = static_cast<int>(std::min<long long>((R + 255) / 256, 148LL * 16));
+    build_masks_kernel<<<blocks, 256, 0, st>>>(idx, d.T, d.k, d.E, reinterpret_cast<uint32_t*>(ws + L.masks), s->err);
+    MOE_TRY(ls_.done());
   }
-  return enqueue_permute(d, L, ws, idx, cnt, off, row_of, token_of, st);
+  return enqueue_permute(d, L, ws, idx, nullptr, cnt, off, row_of, token_of, st);
 }
 
 moe_status moe_get_device_status(void* stream) {

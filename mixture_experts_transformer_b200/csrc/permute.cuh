@@ -6,10 +6,12 @@
 // gm.nn.Gemma4_26B_A4B TransformerConfig); no capacity factor or token
 // dropping is mentioned, so every assignment gets a row.
 //
-//   router_topk_kernel   counts tokens per expert for each chunk of 128 tokens
-//   route_scan_kernel    cnt, off, per-chunk first rows, GEMM tile lists
-//   route_scatter_kernel row_of[t, j] and token_of[row]
-//   gather_rows_kernel   x_perm[row] = x[token_of[row]]
+// Everything derives from the 32-token expert bitmasks mask[c][e] (bit i set
+// when token 32c + i chose expert e):
+//   cnt[e]          = sum_c popc(mask[c][e])
+//   base[c][e]      = off[e] + sum_{c' < c} popc(mask[c'][e])
+//   row of (t, e)   = base[t/32][e] + popc(mask[t/32][e] & ((1 << t%32) - 1))
+// so the scan is one small CTA and the scatter has no loops at all.
 #pragma once
 
 #include "grouped_gemm.cuh"
@@ -17,74 +19,106 @@
 
 namespace moe {
 
+constexpr int kScanThreads = 1024;
+constexpr int kScanSegs = kScanThreads / 128;
+
 struct TileCounts {
   int32_t gateup;
   int32_t down;
 };
 
-// Tokens per expert for each chunk of kTopkChunk tokens of a given idx
-// [T, k] (the same counts router_topk_kernel produces as a side result).
-__global__ void __launch_bounds__(128) chunk_histogram_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
-                                                              int32_t* __restrict__ chunk_cnt, uint32_t* err) {
-  __shared__ int s_cnt[128];
-  if (threadIdx.x < 128) s_cnt[threadIdx.x] = 0;
-  __syncthreads();
-  const int t0 = blockIdx.x * kTopkChunk;
-  const int n = (min(T, t0 + kTopkChunk) - t0) * k;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int e = idx[static_cast<size_t>(t0) * k + i];
+// Bitmasks of a given idx [T, k] (moe_permute's entry; the forward pass gets
+// them from router_topk_kernel). masks must be zero on entry.
+__global__ void build_masks_kernel(const int32_t* __restrict__ idx, int T, int k, int E, uint32_t* __restrict__ masks,
+                                   uint32_t* err) {
+  const int n = T * k;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int t = i / k;
+    const int e = idx[i];
     if (e < 0 || e >= E) {
       atomicOr(err, kErrBadIndex);
       continue;
     }
-    atomicAdd(&s_cnt[e], 1);
+    atomicOr(masks + static_cast<size_t>(t / kMaskTokens) * E + e, 1u << (t & (kMaskTokens - 1)));
   }
-  __syncthreads();
-  if (threadIdx.x < E) chunk_cnt[static_cast<size_t>(blockIdx.x) * E + threadIdx.x] = s_cnt[threadIdx.x];
 }
 
-// One CTA, thread e = expert. chunk_cnt[c][e] (tokens of chunk c routed to e)
-// becomes the first routed row of chunk c's assignments to e. Also writes the
-// tile lists: shared-MLP tiles first (problem 1), then expert tiles (problem 0),
-// expert-major, then column tile, then row tile, so CTAs that run at the same
-// time read the same weight columns and share them through L2.
-__global__ void __launch_bounds__(128) route_scan_kernel(int32_t* __restrict__ chunk_cnt, int nchunks, int T, int E,
-                                                         int F, int S, int D, int32_t* __restrict__ cnt_out,
-                                                         int32_t* __restrict__ off_out, Tile* __restrict__ tiles_gu,
-                                                         Tile* __restrict__ tiles_dn,
-                                                         TileCounts* __restrict__ counts) {
+// One CTA of 1024 threads: thread (e, seg) walks one eighth of the 32-token
+// chunks of expert e. Produces cnt, off, base[c][e] and the tile lists:
+// shared-MLP tiles first (problem 1), then expert tiles (problem 0) expert by
+// expert, column tile, then row tile, so CTAs that run at the same time read
+// the same weight columns and share them through L2.
+__global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t* __restrict__ masks, int nchunks,
+                                                                  int T, int E, int F, int S, int D,
+                                                                  int32_t* __restrict__ base,
+                                                                  int32_t* __restrict__ cnt_out,
+                                                                  int32_t* __restrict__ off_out,
+                                                                  Tile* __restrict__ tiles_gu,
+                                                                  Tile* __restrict__ tiles_dn,
+                                                                  TileCounts* __restrict__ counts) {
+  __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
   __shared__ int s_cnt[128];
-  const int e = threadIdx.x;
-  int c_e = 0;
-  if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = chunk_cnt[static_cast<size_t>(c) * E + e];
-      chunk_cnt[static_cast<size_t>(c) * E + e] = c_e;
-      c_e += v;
-    }
-  }
-  s_cnt[e] = e < E ? c_e : 0;
+  const int e = threadIdx.x & 127;
+  const int seg = threadIdx.x >> 7;
+  const int c0 = static_cast<int>((static_cast<long long>(seg) * nchunks) / kScanSegs);
+  const int c1 = static_cast<int>((static_cast<long long>(seg + 1) * nchunks) / kScanSegs);
+  int part = 0;
+  if (e < E)
+    for (int c = c0; c < c1; ++c) part += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
+  s_seg[seg][e] = part;
   __syncthreads();
-  if (e == 0) {
-    int o = 0, mo = 0;
-    for (int i = 0; i < E; ++i) {
-      s_off[i] = o;
-      s_mtoff[i] = mo;
-      o += s_cnt[i];
-      mo += (s_cnt[i] + kBM - 1) / kBM;
+  if (seg == 0) {
+    int run = 0;
+    for (int s = 0; s < kScanSegs; ++s) {
+      const int v = s_seg[s][e];
+      s_seg[s][e] = run;
+      run += v;
     }
-    s_off[E] = o;
-    s_mtoff[E] = mo;
+    s_cnt[e] = e < E ? run : 0;
   }
   __syncthreads();
-  if (e < E) {
-    cnt_out[e] = c_e;
-    off_out[e] = s_off[e];
-    for (int c = 0; c < nchunks; ++c) chunk_cnt[static_cast<size_t>(c) * E + e] += s_off[e];
+  if (threadIdx.x < 32) {  // exclusive scans over experts, one warp
+    const int lane = threadIdx.x;
+    int carry = 0, mcarry = 0;
+    for (int b = 0; b < 128; b += 32) {
+      const int v = s_cnt[b + lane];
+      const int mv = (v + kBM - 1) / kBM;
+      int inc = v, minc = mv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, inc, o);
+        const int ma = __shfl_up_sync(0xffffffffu, minc, o);
+        if (lane >= o) {
+          inc += a;
+          minc += ma;
+        }
+      }
+      s_off[b + lane] = carry + inc - v;
+      s_mtoff[b + lane] = mcarry + minc - mv;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+      mcarry += __shfl_sync(0xffffffffu, minc, 31);
+    }
+    if (lane == 0) {
+      s_off[E] = carry;
+      s_mtoff[E] = mcarry;
+    }
   }
-  if (e == 0) off_out[E] = s_off[E];
+  __syncthreads();
+  const int c_e = s_cnt[e];
+  if (e < E) {
+    int run = s_off[e] + s_seg[seg][e];
+    for (int c = c0; c < c1; ++c) {
+      base[static_cast<size_t>(c) * E + e] = run;
+      run += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
+    }
+    if (seg == 0) {
+      cnt_out[e] = c_e;
+      off_out[e] = s_off[e];
+    }
+  }
+  if (threadIdx.x == 0) off_out[E] = s_off[E];
 
   const int mt_sh = (T + kBM - 1) / kBM;
   const int nt_gu_sh = (S + 127) / 128;
@@ -92,11 +126,11 @@ __global__ void __launch_bounds__(128) route_scan_kernel(int32_t* __restrict__ c
   const int nt_dn = (D + 255) / 256;
   const int n_sh_gu = nt_gu_sh * mt_sh;
   const int n_sh_dn = nt_dn * mt_sh;
-  for (int i = threadIdx.x; i < n_sh_gu; i += blockDim.x) {
+  for (int i = threadIdx.x; i < n_sh_gu; i += kScanThreads) {
     const int nt = i / mt_sh, m = i % mt_sh;
     tiles_gu[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * 128};
   }
-  for (int i = threadIdx.x; i < n_sh_dn; i += blockDim.x) {
+  for (int i = threadIdx.x; i < n_sh_dn; i += kScanThreads) {
     const int nt = i / mt_sh, m = i % mt_sh;
     tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * 256};
   }
@@ -104,58 +138,56 @@ __global__ void __launch_bounds__(128) route_scan_kernel(int32_t* __restrict__ c
     const int mt = (c_e + kBM - 1) / kBM;
     const int base_gu = n_sh_gu + s_mtoff[e] * nt_gu;
     const int base_dn = n_sh_dn + s_mtoff[e] * nt_dn;
-    for (int nt = 0; nt < nt_gu; ++nt)
-      for (int m = 0; m < mt; ++m)
-        tiles_gu[base_gu + nt * mt + m] = Tile{e, s_off[e] + m * kBM, min(kBM, c_e - m * kBM), nt * 128};
-    for (int nt = 0; nt < nt_dn; ++nt)
-      for (int m = 0; m < mt; ++m)
-        tiles_dn[base_dn + nt * mt + m] = Tile{e, s_off[e] + m * kBM, min(kBM, c_e - m * kBM), nt * 256};
+    for (int i = seg; i < nt_gu * mt; i += kScanSegs) {
+      const int nt = i / mt, m = i % mt;
+      tiles_gu[base_gu + i] = Tile{e, s_off[e] + m * kBM, min(kBM, c_e - m * kBM), nt * 128};
+    }
+    for (int i = seg; i < nt_dn * mt; i += kScanSegs) {
+      const int nt = i / mt, m = i % mt;
+      tiles_dn[base_dn + i] = Tile{e, s_off[e] + m * kBM, min(kBM, c_e - m * kBM), nt * 256};
+    }
   }
-  if (e == 0) {
+  if (threadIdx.x == 0) {
     counts->gateup = n_sh_gu + s_mtoff[E] * nt_gu;
     counts->down = n_sh_dn + s_mtoff[E] * nt_dn;
   }
 }
 
-// CTA c, thread e: walk chunk c's tokens in order and hand out expert e's rows.
-__global__ void __launch_bounds__(128) route_scatter_kernel(const int32_t* __restrict__ idx,
-                                                            const int32_t* __restrict__ chunk_first_row, int T,
-                                                            int k, int E, int32_t* __restrict__ row_of,
-                                                            int32_t* __restrict__ token_of) {
-  const int e = threadIdx.x;
-  const int c = blockIdx.x;
-  if (e >= E) return;
-  int r = chunk_first_row[static_cast<size_t>(c) * E + e];
-  const int t_end = min(T, (c + 1) * kTopkChunk);
-  for (int t = c * kTopkChunk; t < t_end; ++t) {
-    const int32_t* it = idx + static_cast<size_t>(t) * k;
-    for (int j = 0; j < k; ++j) {
-      if (__ldg(it + j) == e) {
-        row_of[static_cast<size_t>(t) * k + j] = r;
-        token_of[r] = t;
-        ++r;
-        break;
-      }
+// One warp per (token, slot): its routed row from the bitmasks; lane 0 writes
+// row_of / token_of, and (when x is given) the warp copies x[t] into
+// x_perm[row] with 16-byte vectors.
+__global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __restrict__ idx,
+                                                            const uint32_t* __restrict__ masks,
+                                                            const int32_t* __restrict__ base, int T, int k, int E,
+                                                            int D, const __nv_bfloat16* __restrict__ x,
+                                                            int32_t* __restrict__ row_of,
+                                                            int32_t* __restrict__ token_of,
+                                                            __nv_bfloat16* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const long long R = static_cast<long long>(T) * k;
+  for (long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); a < R;
+       a += static_cast<long long>(gridDim.x) * 8) {
+    const int t = static_cast<int>(a / k);
+    const int e = __ldg(idx + a);
+    if (e < 0 || e >= E) continue;  // reported by build_masks_kernel
+    const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
+    const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
+    const int row = __ldg(base + cw) + __popc(below);
+    if (lane == 0) {
+      row_of[a] = row;
+      token_of[row] = t;
+    }
+    if (x) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * D);
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(row) * D);
+      for (int i = lane; i < (D >> 3); i += 32) dst[i] = __ldg(src + i);
     }
   }
 }
 
-// x_perm[row, :] = x[token_of[row], :]; one warp per row, 16-byte vectors.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
-                                                          const int32_t* __restrict__ token_of, int R, int D,
-                                                          __nv_bfloat16* __restrict__ xp) {
-  const int lane = threadIdx.x & 31;
-  const int nvec = D >> 3;
-  for (int row = blockIdx.x * 8 + (threadIdx.x >> 5); row < R; row += gridDim.x * 8) {
-    const int t = __ldg(token_of + row);
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * D);
-    uint4* dst = reinterpret_cast<uint4*>(xp + static_cast<size_t>(row) * D);
-    for (int i = lane; i < nvec; i += 32) dst[i] = __ldg(src + i);
-  }
-}
-
 // out[t] = RNE_bf16(s[t] + w[t,0] y[row_of[t,0]] + ... + w[t,k-1] y[row_of[t,k-1]]),
-// accumulated in fp32 in slot order (deterministic, no atomics).
+// accumulated in fp32 in slot order (deterministic, no atomics). Grid (T,
+// dsplit): CTA (t, q) handles the q-th slice of the row's 8-column vectors.
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ s, const __nv_bfloat16* __restrict__ y,
                                                      const int32_t* __restrict__ row_of,
                                                      const float* __restrict__ w, int T, int k, int D,
@@ -169,11 +201,27 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   }
   __syncthreads();
   const int nvec = D >> 3;
-  for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+  const int per = (nvec + gridDim.y - 1) / gridDim.y;
+  const int v0 = blockIdx.y * per, v1 = min(nvec, v0 + per);
+  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
     const float4* sp = reinterpret_cast<const float4*>(s + static_cast<size_t>(t) * D) + 2 * v;
     const float4 s0 = sp[0], s1 = sp[1];
     float acc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    for (int j = 0; j < k; ++j) {
+    int j = 0;
+    for (; j + 4 <= k; j += 4) {  // four rows' loads in flight, accumulated in slot order
+      uint4 yv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        yv[u] = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j + u]) * D) + v);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(&yv[u]);
+        const float wj = s_w[j + u];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, __bfloat162float(yb[i]), acc[i]);
+      }
+    }
+    for (; j < k; ++j) {
       const uint4 yv = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j]) * D) + v);
       const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(&yv);
       const float wj = s_w[j];
@@ -192,11 +240,6 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
       op[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
   }
-}
-
-// Copy the routing of each token into caller buffers (debug outputs).
-__global__ void copy_i32_kernel(const int32_t* __restrict__ a, int32_t* __restrict__ b, int n) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) b[i] = a[i];
 }
 
 // A kernel that waits, bounded, on a barrier nothing completes: the failure

@@ -18,11 +18,12 @@ from oracle import moe_oracle as mo
 OUT_TOL = 1e-2
 # At reduced test shapes the routed branch carries a larger share of the output
 # than in the real block (fewer, narrower experts), and the one deliberate
-# precision loss of the path - the bf16 storage of the GeGLU rows h and of the
-# expert outputs y, each rounded to nearest even (relative error <= 2^-8) - can
+# precision loss of the path - the bf16 storage of the GeGLU rows (routed h and
+# shared hs) and of the expert outputs y, each rounded to nearest even
+# (relative error <= 2^-8) - can
 # approach 1e-2 * RMS by itself. There the tolerance is derived from that
-# arithmetic: the test evaluates the oracle's formula with h and y rounded to
-# bf16 (float64 otherwise) to measure the rounding's own cost e_bf16, and allows
+# arithmetic: the test evaluates the oracle's formula with h, hs and y rounded
+# to bf16 (float64 otherwise) to measure the rounding's own cost e_bf16, and allows
 # 1.25 * e_bf16 plus 2e-3 * RMS for fp32 accumulation and the tanh
 # approximation, or 1e-2 * RMS, whichever is larger.
 BF16_SLACK = 1.25
@@ -97,10 +98,12 @@ def _rne_bf16_f64(a):
 
 
 def bf16_storage_cost(xs, w_host, idx, wts):
-    """max |out(h, y rounded to bf16) - out(exact)| for the given routing (CPU, float64)."""
+    """max |out(h, y, hs rounded to bf16) - out(exact)| for the given routing (CPU, float64)."""
     x = mo.f64(xs)
-    exact = np.zeros((x.shape[0], x.shape[1]))
-    rounded = np.zeros_like(exact)
+    hs = mo.geglu_hidden(x, w_host.sg, w_host.su)
+    sd = mo.f64(w_host.sd)
+    exact = hs @ sd
+    rounded = _rne_bf16_f64(hs) @ sd  # the shared hidden rows are stored in bf16 too
     for e in np.unique(idx):
         tok, slot = np.nonzero(idx == e)
         h = mo.geglu_hidden(x[tok], w_host.wg[e], w_host.wu[e])
