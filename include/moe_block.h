@@ -200,14 +200,16 @@ moe_status moe_debug_timeout_probe(int timeout_us, void* stream);
 moe_status moe_block_forward_hostio(const moe_params* p, const void* x_host, void* out_host, void* stream);
 
 /*
- * Per-kernel timing. After moe_profile_begin(), every kernel this thread
- * enqueues is bracketed by two CUDA events recorded on its stream.
+ * Per-kernel timing. After moe_profile_begin(kernel_mask), every kernel this
+ * thread enqueues whose id bit is set in kernel_mask is bracketed by two CUDA
+ * events recorded on its stream (an event between two kernels also ends their
+ * launch overlap, so time the whole step with a narrow mask).
  * moe_profile_end() waits for those events, writes per kernel id the summed
  * milliseconds and the number of launches into total_ms[0..n) and
  * launches[0..n), stops recording and returns the number of kernel ids.
  * moe_kernel_name(id) names a kernel id (NULL past the last one).
  */
-moe_status moe_profile_begin(void);
+moe_status moe_profile_begin(uint32_t kernel_mask);
 int moe_profile_end(float* total_ms, int* launches, int n);
 const char* moe_kernel_name(int id);
 

@@ -73,7 +73,7 @@ EXPORTS = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_launch_count": (ctypes.c_int, []),
     "moe_block_forward_hostio": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp, _vp]),
-    "moe_profile_begin": (ctypes.c_int, []),
+    "moe_profile_begin": (ctypes.c_int, [ctypes.c_uint32]),
     "moe_profile_end": (ctypes.c_int, [_vp, _vp, ctypes.c_int]),
     "moe_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -238,8 +238,27 @@ def moe_block_forward_hostio(p: MoeParams, x_host, out_host, stream=None) -> int
     return lib().moe_block_forward_hostio(ctypes.byref(p), ptr(x_host), ptr(out_host), stream_handle(stream))
 
 
-def moe_profile_begin() -> int:
-    return lib().moe_profile_begin()
+def kernel_ids() -> dict:
+    """{kernel name: id} of the library's kernels."""
+    out, i = {}, 0
+    while True:
+        n = lib().moe_kernel_name(i)
+        if n is None:
+            return out
+        out[n.decode()] = i
+        i += 1
+
+
+def moe_profile_begin(kernels=None) -> int:
+    """Record events around the named kernels (all when None)."""
+    if kernels is None:
+        mask = 0xFFFFFFFF
+    else:
+        ids = kernel_ids()
+        mask = 0
+        for k in kernels:
+            mask |= 1 << ids[k]
+    return lib().moe_profile_begin(mask)
 
 
 def moe_profile_end(n: int = 32) -> dict:

@@ -121,6 +121,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above touched only this CTA's shared memory and TMEM; the tile
+  // list, A and the outputs belong to the previous kernels
+  pdl_wait_then_release();
   const int num_tiles = *P.num_tiles;
 
   if (warp == 0) {

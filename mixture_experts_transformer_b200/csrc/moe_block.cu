@@ -230,6 +230,7 @@ struct ProfRecord {
   cudaEvent_t start, stop;
 };
 thread_local bool t_profiling = false;
+thread_local uint32_t t_profile_mask = 0;
 thread_local std::vector<ProfRecord> t_records;
 thread_local std::vector<cudaEvent_t> t_event_pool;
 
@@ -250,21 +251,40 @@ struct LaunchScope {
   int id;
   cudaEvent_t a = nullptr;
   LaunchScope(int id_, cudaStream_t st_) : st(st_), id(id_) {
-    if (t_profiling) {
+    if (t_profiling && ((t_profile_mask >> id) & 1u)) {
       a = pooled_event();
       cudaEventRecord(a, st);
     }
   }
-  moe_status done() {
+  moe_status done(cudaError_t launch_err) {
     ++t_launches;
     if (t_profiling && a) {
       cudaEvent_t b = pooled_event();
       cudaEventRecord(b, st);
       t_records.push_back(ProfRecord{id, a, b});
     }
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
 };
+
+// Every kernel is launched with programmatic stream serialization: it may
+// start while its predecessor drains, and waits (griddepcontrol.wait) before
+// touching memory, so launch latency and prologues overlap the previous
+// kernel's tail.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 #define MOE_TRY(expr)                   \
   do {                                  \
@@ -316,15 +336,15 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
   const dim3 g1((d.T + kRouterTokens - 1) / kRouterTokens, L.nsplit);
   {
     LaunchScope ls_(kKRouterLogits, st);
-    router_logits_kernel<<<g1, kRouterThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+    const cudaError_t le_ = launch_k(router_logits_kernel, g1, kRouterThreads, 0, st, static_cast<const __nv_bfloat16*>(x),
                                                         static_cast<const __nv_bfloat16*>(wr), partial, masks, d.T,
                                                         d.D, d.E, L.nsplit);
-    MOE_TRY(ls_.done());
+    MOE_TRY(ls_.done(le_));
   }
   LaunchScope ls_(kKRouterTopk, st);
-  router_topk_kernel<<<(d.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st>>>(partial, bias, d.T, d.E,
+  const cudaError_t le_ = launch_k(router_topk_kernel, (d.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
                                                                                      L.nsplit, d.k, idx, w, masks);
-  return ls_.done();
+  return ls_.done(le_);
 }
 
 // Scan of the bitmasks, then the scatter (and, with x, the gather into x_perm).
@@ -334,19 +354,19 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   {
     LaunchScope ls_(kKRouteScan, st);
-    route_scan_kernel<<<1, kScanThreads, 0, st>>>(masks, L.nchunks, d.T, d.E, d.F, d.S, d.D, base, cnt, off,
+    const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S, d.D, base, cnt, off,
                                                   reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                                   reinterpret_cast<Tile*>(ws + L.tiles_dn),
                                                   reinterpret_cast<TileCounts*>(ws + L.counts));
-    MOE_TRY(ls_.done());
+    MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
   const int blocks = static_cast<int>(std::min<long long>((R + 7) / 8, 148LL * 64));
   LaunchScope ls_(kKRouteScatter, st);
-  route_scatter_kernel<<<blocks, 256, 0, st>>>(idx, masks, base, d.T, d.k, d.E, d.D,
+  const cudaError_t le_ = launch_k(route_scatter_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E, d.D,
                                                static_cast<const __nv_bfloat16*>(x), row_of, token_of,
                                                reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm));
-  return ls_.done();
+  return ls_.done(le_);
 }
 
 moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, uint8_t* ws, DeviceState* s,
@@ -384,8 +404,8 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   const int grid_gu = std::min(s->sm_count, L.max_tiles_gu);
   {
   LaunchScope ls_(kKGemmGateUp, st);
-  grouped_gemm_kernel<true><<<grid_gu, kGemmThreads, kGemmSmemBytes, st>>>(gu);
-  MOE_TRY(ls_.done());
+  const cudaError_t le_ = launch_k(grouped_gemm_kernel<true>, grid_gu, kGemmThreads, kGemmSmemBytes, st, gu);
+  MOE_TRY(ls_.done(le_));
   }
 
   // down: experts -> y (bf16), shared -> s (fp32)
@@ -405,16 +425,16 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   const int grid_dn = std::min(s->sm_count, L.max_tiles_dn);
   {
   LaunchScope ls_(kKGemmDown, st);
-  grouped_gemm_kernel<false><<<grid_dn, kGemmThreads, kGemmSmemBytes, st>>>(dn);
-  MOE_TRY(ls_.done());
+  const cudaError_t le_ = launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn);
+  MOE_TRY(ls_.done(le_));
   }
 
   {
   LaunchScope ls_(kKCombine, st);
   const int dsplit = std::max(1, std::min(4, (2 * s->sm_count) / std::max(1, d.T)));
-  combine_kernel<<<dim3(d.T, dsplit), 128, 0, st>>>(sbuf, y, row_of, w, d.T, d.k, d.D,
+  const cudaError_t le_ = launch_k(combine_kernel, dim3(d.T, dsplit), 128, 0, st, sbuf, y, row_of, w, d.T, d.k, d.D,
                                                     static_cast<__nv_bfloat16*>(p->out), p->out_f32);
-  MOE_TRY(ls_.done());
+  MOE_TRY(ls_.done(le_));
   }
 
   if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -540,8 +560,8 @@ moe_status moe_permute(const moe_params* p, const int32_t* idx, int32_t* cnt, in
     LaunchScope ls_(kKBuildMasks, st);
     const long long R = static_cast<long long>(d.T) * d.k;
     const int blocks = static_cast<int>(std::min<long long>((R + 255) / 256, 148LL * 16));
-    build_masks_kernel<<<blocks, 256, 0, st>>>(idx, d.T, d.k, d.E, reinterpret_cast<uint32_t*>(ws + L.masks), s->err);
-    MOE_TRY(ls_.done());
+    const cudaError_t le_ = launch_k(build_masks_kernel, blocks, 256, 0, st, idx, d.T, d.k, d.E, reinterpret_cast<uint32_t*>(ws + L.masks), s->err);
+    MOE_TRY(ls_.done(le_));
   }
   return enqueue_permute(d, L, ws, idx, nullptr, cnt, off, row_of, token_of, st);
 }
@@ -566,9 +586,9 @@ moe_status moe_debug_timeout_probe(int timeout_us, void* stream) {
   MOE_TRY(device_state(&s));
   {
   LaunchScope ls_(kKTimeoutProbe, static_cast<cudaStream_t>(stream));
-  timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+  const cudaError_t le_ = launch_k(timeout_probe_kernel, 1, 32, 0, static_cast<cudaStream_t>(stream), 
       s->err, static_cast<unsigned long long>(timeout_us) * 1000ull);
-  return ls_.done();
+  return ls_.done(le_);
   }
 }
 
@@ -608,7 +628,8 @@ moe_status moe_block_forward_hostio(const moe_params* p, const void* x_host, voi
   return MOE_OK;
 }
 
-moe_status moe_profile_begin(void) {
+moe_status moe_profile_begin(uint32_t kernel_mask) {
+  t_profile_mask = kernel_mask;
   for (const ProfRecord& r : t_records) {
     t_event_pool.push_back(r.start);
     t_event_pool.push_back(r.stop);

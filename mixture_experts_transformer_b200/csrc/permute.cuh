@@ -31,6 +31,7 @@ struct TileCounts {
 // them from router_topk_kernel). masks must be zero on entry.
 __global__ void build_masks_kernel(const int32_t* __restrict__ idx, int T, int k, int E, uint32_t* __restrict__ masks,
                                    uint32_t* err) {
+  pdl_wait_then_release();
   const int n = T * k;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     const int t = i / k;
@@ -60,6 +61,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
   __shared__ int s_cnt[128];
+  pdl_wait_then_release();
   const int e = threadIdx.x & 127;
   const int seg = threadIdx.x >> 7;
   const int c0 = static_cast<int>((static_cast<long long>(seg) * nchunks) / kScanSegs);
@@ -163,6 +165,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
                                                             int32_t* __restrict__ row_of,
                                                             int32_t* __restrict__ token_of,
                                                             __nv_bfloat16* __restrict__ x_perm) {
+  pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const long long R = static_cast<long long>(T) * k;
   for (long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); a < R;
@@ -194,6 +197,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                                      __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32) {
   __shared__ int s_row[128];
   __shared__ float s_w[128];
+  pdl_wait_then_release();
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < k; j += blockDim.x) {
     s_row[j] = row_of[static_cast<size_t>(t) * k + j];
@@ -247,6 +251,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 __global__ void timeout_probe_kernel(uint32_t* err, unsigned long long timeout_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
+  pdl_wait_then_release();
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     abort_flag = 0;

@@ -80,6 +80,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ------------------------------------------------------- dependent launch
+
+// Programmatic dependent launch: wait until the previous kernel in the stream
+// has completed and its writes are visible (a no-op without the launch
+// attribute), then let the next kernel start launching. Every kernel of the
+// library calls this before its first global-memory access, so overlap with
+// the neighbouring kernels never reaches data.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const __n
   __shared__ __align__(16) float xs[kRouterKChunk][kRouterTokens];
   __shared__ __align__(16) float ws[kRouterKChunk][128];
 
+  pdl_wait_then_release();
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int tg = lane >> 3, eg = lane & 7;
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) router_topk_kernel(const floa
                                                                      int nsplit, int k, int32_t* __restrict__ idx,
                                                                      float* __restrict__ wts,
                                                                      uint32_t* __restrict__ masks) {
+  pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
   if (t >= T) return;
