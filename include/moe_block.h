@@ -213,6 +213,31 @@ moe_status moe_profile_begin(uint32_t kernel_mask);
 int moe_profile_end(float* total_ms, int* launches, int n);
 const char* moe_kernel_name(int id);
 
+/*
+ * moe_route without any device allocation (the pages have no counterpart; it
+ * exists for callers of this library that are not allowed to allocate device
+ * memory: applications whose memory is owned by their own allocator or
+ * reserved up front, which forbid libraries to call cudaMalloc behind their
+ * back, and runtimes whose allocation calls would stall or fail mid-run).
+ *
+ * Same arguments, kernels and results as moe_route (idx and w are caller
+ * memory; the workspace fields of p are ignored). Its scratch - the split-K
+ * partial logits and the token-expert bitmasks - lives in a fixed 4 MiB
+ * __device__ array inside the library, which every GPU that loads the library
+ * holds until the process exits. T is limited to 4096 tokens (and the scratch
+ * must fit: the split of the reduction is narrowed when needed); a larger
+ * batch returns MOE_ERR_WORKSPACE before anything is enqueued. No cudaMalloc,
+ * cudaFree or allocating library routine is called.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) once for that device; make that first call before
+ * any stream capture. Every call on a device shares the one array, and a call
+ * overwrites what the previous call left there: calls that may overlap on the
+ * GPU (different streams, or different host threads) race and must be
+ * serialised by the caller.
+ */
+moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* stream);
+
 /* Human-readable name of a status code. */
 const char* moe_status_string(moe_status s);
 

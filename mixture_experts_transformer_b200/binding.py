@@ -76,6 +76,7 @@ EXPORTS = {
     "moe_profile_begin": (ctypes.c_int, [ctypes.c_uint32]),
     "moe_profile_end": (ctypes.c_int, [_vp, _vp, ctypes.c_int]),
     "moe_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_route_noalloc": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp, _vp]),
 }
 
 _lib = None
@@ -271,3 +272,8 @@ def moe_profile_end(n: int = 32) -> dict:
         if cnt[i]:
             out[lib().moe_kernel_name(i).decode()] = (float(ms[i]), int(cnt[i]))
     return out
+
+
+def moe_route_noalloc(p: MoeParams, idx, w, stream=None) -> int:
+    """moe_route with its scratch in the library's fixed device array (no allocation)."""
+    return lib().moe_route_noalloc(ctypes.byref(p), ptr(idx), ptr(w), stream_handle(stream))

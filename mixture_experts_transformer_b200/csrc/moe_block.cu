@@ -449,6 +449,36 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
 }  // namespace
 }  // namespace moe
 
+namespace moe {
+namespace {
+
+// Scratch of moe_route_noalloc: one fixed array per device that loads this
+// library, held until the process exits. It carries the router's split-K
+// partial logits and the 32-token expert bitmasks of a single call.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr int kNoAllocMaxTokens = 4096;
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+uint8_t* g_noalloc_base[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of this device's scratch array, looked up once per device
+// (the host-side symbol is only a stand-in and must never reach a kernel).
+moe_status noalloc_base(uint8_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_base[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return MOE_ERR_CUDA;
+    g_noalloc_base[dev] = static_cast<uint8_t*>(ptr);
+  }
+  *out = g_noalloc_base[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
 using namespace moe;
 
 extern "C" {
@@ -661,5 +691,32 @@ int moe_profile_end(float* total_ms, int* launches, int n) {
 }
 
 const char* moe_kernel_name(int id) { return (id >= 0 && id < kKCount) ? kKernelNames[id] : nullptr; }
+
+moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* stream) {
+  t_launches = 0;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  const Dims d = dims_of(p);
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  if (d.T == 0) return MOE_OK;
+  if (d.T > kNoAllocMaxTokens) return MOE_ERR_WORKSPACE;
+  if (!p->x || !p->w_router || !idx || !w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned4(idx) || !aligned4(w)) return MOE_ERR_ALIGNMENT;
+  if (p->router_bias && !aligned4(p->router_bias)) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  uint8_t* scratch = nullptr;
+  MOE_TRY(noalloc_base(&scratch));
+  // Same kernels and split of the reduction as moe_route, with the partial
+  // logits and bitmasks placed in the fixed array; the split shrinks only if
+  // the partials would not fit (the bitmasks are cleared by the router kernel).
+  Layout L = make_layout(d);
+  const size_t mask_bytes = align_up(static_cast<size_t>(L.nchunks) * d.E * 4, kAlign);
+  auto partial_bytes = [&](int ns) { return align_up(static_cast<size_t>(ns) * d.T * d.E * 4, kAlign); };
+  while (L.nsplit > 1 && partial_bytes(L.nsplit) + mask_bytes > kNoAllocScratchBytes) --L.nsplit;
+  if (partial_bytes(L.nsplit) + mask_bytes > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+  L.partial = 0;
+  L.masks = partial_bytes(L.nsplit);
+  return enqueue_route(d, L, scratch, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream));
+}
 
 }  // extern "C"
