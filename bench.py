@@ -189,10 +189,11 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def csrc_digest() -> str:
+def source_digest(files) -> str:
+    """Hash of the kernel source files an ncu capture was taken on."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_transformer_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -200,14 +201,14 @@ def csrc_digest() -> str:
 
 def ncu_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         table = json.load(f)
     ent = table.get(f"{kernel}@{workload}")
-    if not ent or ent.get("csrc") != csrc_digest():
+    if not ent or ent.get("digest") != source_digest(ent.get("files", [])):
         return None
     return ent.get("bytes_per_launch")
 
