@@ -238,6 +238,98 @@ const char* moe_kernel_name(int id);
  */
 moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* stream);
 
+/* ------------------------------------------------------------------ NVFP4
+ *
+ * The NVFP4 variant follows the checkpoint's quantisation_config
+ * (G4-MeroMero-26B-A4B-NVFP4 config.json, config_groups.group_0): every
+ * expert and shared Linear holds e2m1 values in groups of 16 along its input
+ * dimension K with one float8_e4m3 scale per group and one fp32 tensor scale
+ * ("tensor_group"); weights are static, input activations are quantised per
+ * call under a calibrated tensor scale ("dynamic": "local", static_minmax);
+ * the router stays bf16 ("ignore": layers.N.router.proj).
+ *
+ * Quantisation of a group under tensor scale G, in fp32 with IEEE
+ * round-to-nearest operations:
+ *   s = e4m3_satfinite(RN(RN(amax16 / 6) * G)); q_i = e2m1_satfinite(RN(x_i * RN(G / s)))
+ *   (s = 0 makes the group 0); value x^_i = e2m1(q_i) * s / G; weights use G = 448*6/amax.
+ *
+ * Storage of one [K, N] Linear (or G of them, experts stacked):
+ *   q  [G][N][K/2] bytes: e2m1 codes, K-major, element 2j of a row in the low
+ *      nibble of byte j;
+ *   sf [G][ceil(N/128)][K/64][512] bytes: the group scales of rows 128a..128a+127
+ *      and K range 64b..64b+63 form one 512-byte atom, row r, 16-group c (0..3)
+ *      at byte 16*(r%32) + 4*(r/32) + c; rows past N hold scale 0;
+ *   g  [G] fp32 tensor scales.
+ */
+typedef struct moe_nvfp4_linear {
+  const uint8_t* q;
+  const uint8_t* sf;
+  const float* g;
+} moe_nvfp4_linear;
+
+/* Sizes of q and sf for G groups of [K, N] (K a multiple of 64, N of 64). */
+moe_status moe_nvfp4_weight_bytes(int groups, int K, int N, size_t* q_bytes, size_t* sf_bytes);
+
+/*
+ * Quantise bf16 weights w [groups][K][N] (N contiguous: exactly the layout the
+ * bf16 block takes) into q, sf and g (caller-owned device buffers of the sizes
+ * above). Deterministic; enqueued on stream.
+ */
+moe_status moe_nvfp4_quantize_weight(const void* w, int groups, int K, int N, uint8_t* q, uint8_t* sf, float* g,
+                                     void* stream);
+
+/*
+ * Quantise activation rows x [rows][K] bf16 under tensor scale g into
+ * q [rows][K/2] and sf [ceil(rows/128)][K/64][512] (the same formats; a
+ * standalone entry to the quantiser the NVFP4 block applies to x).
+ */
+moe_status moe_nvfp4_quantize_act(const void* x, int rows, int K, float g, uint8_t* q, uint8_t* sf, void* stream);
+
+/*
+ * Parameters of one NVFP4 block. Dims, x, w_router, router_bias, out, out_f32,
+ * idx_out, w_out, cnt_out and workspace as in moe_params (num_experts, the
+ * shared width and embed_dim multiples of 128 are not needed; all three dims
+ * multiples of 64). g_x, g_h, g_hs: static tensor scales of the block input,
+ * the routed GeGLU rows and the shared GeGLU rows. rms_norm_out = 1 writes
+ * out = y / sqrt(mean(y^2) + 1e-6) of the block output y (no learned scale):
+ * the inter-block norm of a stack of blocks.
+ */
+typedef struct moe_nvfp4_params {
+  int T;
+  int top_k_experts;
+  int embed_dim;
+  int num_experts;
+  int expert_dim;
+  int hidden_dim;
+  const void* x;
+  const void* w_router;
+  const float* router_bias;
+  moe_nvfp4_linear wg, wu, wd;  /* G = num_experts */
+  moe_nvfp4_linear sg, su, sd;  /* G = 1 */
+  float g_x, g_h, g_hs;
+  int rms_norm_out;
+  void* out;
+  float* out_f32;
+  int32_t* idx_out;
+  float* w_out;
+  int32_t* cnt_out;
+  void* workspace;
+  size_t workspace_bytes;
+} moe_nvfp4_params;
+
+size_t moe_nvfp4_workspace_bytes(const moe_nvfp4_params* p);
+
+/* One NVFP4 block forward pass (router bf16, expert and shared Linears NVFP4). */
+moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream);
+
+/*
+ * Calibration observer for the NVFP4 activation scales: runs the bf16 block on
+ * p (which must carry a caller workspace) and writes amax[0] = max |x|,
+ * amax[1] = max |h| over the routed GeGLU rows, amax[2] = max |hs| over the
+ * shared GeGLU rows (device fp32 [3]). The tensor scales are 448*6/amax.
+ */
+moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream);
+
 /* Human-readable name of a status code. */
 const char* moe_status_string(moe_status s);
 

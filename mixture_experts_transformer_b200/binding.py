@@ -277,3 +277,85 @@ def moe_profile_end(n: int = 32) -> dict:
 def moe_route_noalloc(p: MoeParams, idx, w, stream=None) -> int:
     """moe_route with its scratch in the library's fixed device array (no allocation)."""
     return lib().moe_route_noalloc(ctypes.byref(p), ptr(idx), ptr(w), stream_handle(stream))
+
+
+# ----------------------------------------------------------------- NVFP4
+
+
+class MoeNvfp4Linear(ctypes.Structure):
+    _fields_ = [("q", _vp), ("sf", _vp), ("g", _vp)]
+
+
+class MoeNvfp4Params(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int),
+        ("top_k_experts", ctypes.c_int),
+        ("embed_dim", ctypes.c_int),
+        ("num_experts", ctypes.c_int),
+        ("expert_dim", ctypes.c_int),
+        ("hidden_dim", ctypes.c_int),
+        ("x", _vp),
+        ("w_router", _vp),
+        ("router_bias", _vp),
+        ("wg", MoeNvfp4Linear),
+        ("wu", MoeNvfp4Linear),
+        ("wd", MoeNvfp4Linear),
+        ("sg", MoeNvfp4Linear),
+        ("su", MoeNvfp4Linear),
+        ("sd", MoeNvfp4Linear),
+        ("g_x", ctypes.c_float),
+        ("g_h", ctypes.c_float),
+        ("g_hs", ctypes.c_float),
+        ("rms_norm_out", ctypes.c_int),
+        ("out", _vp),
+        ("out_f32", _vp),
+        ("idx_out", _vp),
+        ("w_out", _vp),
+        ("cnt_out", _vp),
+        ("workspace", _vp),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+EXPORTS.update(
+    {
+        "moe_nvfp4_weight_bytes": (
+            ctypes.c_int,
+            [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)],
+        ),
+        "moe_nvfp4_quantize_weight": (
+            ctypes.c_int,
+            [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp, _vp],
+        ),
+        "moe_nvfp4_quantize_act": (ctypes.c_int, [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_float, _vp, _vp, _vp]),
+        "moe_nvfp4_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeNvfp4Params)]),
+        "moe_block_forward_nvfp4": (ctypes.c_int, [ctypes.POINTER(MoeNvfp4Params), _vp]),
+        "moe_nvfp4_calibrate": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp]),
+    }
+)
+
+
+def moe_nvfp4_weight_bytes(groups: int, K: int, N: int) -> tuple[int, int]:
+    q, sf = ctypes.c_size_t(), ctypes.c_size_t()
+    check(lib().moe_nvfp4_weight_bytes(groups, K, N, ctypes.byref(q), ctypes.byref(sf)), "moe_nvfp4_weight_bytes")
+    return q.value, sf.value
+
+
+def moe_nvfp4_quantize_weight(w, groups, K, N, q, sf, g, stream=None) -> int:
+    return lib().moe_nvfp4_quantize_weight(ptr(w), groups, K, N, ptr(q), ptr(sf), ptr(g), stream_handle(stream))
+
+
+def moe_nvfp4_quantize_act(x, rows, K, g, q, sf, stream=None) -> int:
+    return lib().moe_nvfp4_quantize_act(ptr(x), rows, K, float(g), ptr(q), ptr(sf), stream_handle(stream))
+
+
+def moe_nvfp4_workspace_bytes(p: MoeNvfp4Params) -> int:
+    return lib().moe_nvfp4_workspace_bytes(ctypes.byref(p))
+
+
+def moe_block_forward_nvfp4(p: MoeNvfp4Params, stream=None) -> int:
+    return lib().moe_block_forward_nvfp4(ctypes.byref(p), stream_handle(stream))
+
+
+def moe_nvfp4_calibrate(p: MoeParams, amax, stream=None) -> int:
+    return lib().moe_nvfp4_calibrate(ctypes.byref(p), ptr(amax), stream_handle(stream))

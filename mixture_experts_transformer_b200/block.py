@@ -95,3 +95,114 @@ def workspace_for(dims: Dims, T: int, top_k: int = B.TOP_K, device="cuda") -> tu
     p = B.make_params(T, top_k=top_k, dims=dims)
     lay = B.moe_workspace_layout(p)
     return torch.empty(lay.total_bytes, dtype=torch.uint8, device=device), lay
+
+
+# ----------------------------------------------------------------- NVFP4
+
+
+@dataclasses.dataclass
+class Nvfp4Linear:
+    """One quantised Linear stack on the device: codes, scale atoms, tensor scales."""
+
+    q: torch.Tensor
+    sf: torch.Tensor
+    g: torch.Tensor
+    groups: int
+    K: int
+    N: int
+
+    def struct(self) -> B.MoeNvfp4Linear:
+        return B.MoeNvfp4Linear(self.q.data_ptr(), self.sf.data_ptr(), self.g.data_ptr())
+
+
+def quantize_linear(w: torch.Tensor, stream=None) -> Nvfp4Linear:
+    """w [G][K][N] (or [K][N]) bf16 on the device -> NVFP4 (the library's quantiser)."""
+    w3 = w if w.dim() == 3 else w.unsqueeze(0)
+    G, K, N = w3.shape
+    qb, sfb = B.moe_nvfp4_weight_bytes(G, K, N)
+    q = torch.empty(qb, dtype=torch.uint8, device=w.device)
+    sf = torch.empty(sfb, dtype=torch.uint8, device=w.device)
+    g = torch.empty(G, dtype=torch.float32, device=w.device)
+    B.check(B.moe_nvfp4_quantize_weight(w3, G, K, N, q, sf, g, stream), "moe_nvfp4_quantize_weight")
+    return Nvfp4Linear(q, sf, g, G, K, N)
+
+
+@dataclasses.dataclass
+class Nvfp4Weights:
+    dims: Dims
+    w_router: torch.Tensor
+    wg: Nvfp4Linear
+    wu: Nvfp4Linear
+    wd: Nvfp4Linear
+    sg: Nvfp4Linear
+    su: Nvfp4Linear
+    sd: Nvfp4Linear
+
+
+def quantize_block(dw: DeviceWeights, stream=None) -> Nvfp4Weights:
+    return Nvfp4Weights(
+        dw.dims,
+        dw.w_router,
+        *(quantize_linear(t, stream) for t in (dw.wg, dw.wu, dw.wd, dw.sg, dw.su, dw.sd)),
+    )
+
+
+def forward_nvfp4(
+    nw: Nvfp4Weights,
+    x: torch.Tensor,
+    act_scales,
+    *,
+    top_k: int = B.TOP_K,
+    router_bias: torch.Tensor | None = None,
+    rms_norm_out: bool = False,
+    debug: bool = False,
+    workspace: torch.Tensor | None = None,
+    out: torch.Tensor | None = None,
+    stream=None,
+) -> BlockResult:
+    """One NVFP4 block; act_scales = (g_x, g_h, g_hs)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, nw.dims.embed_dim), dtype=torch.bfloat16, device=x.device)
+    res = BlockResult(out=out)
+    if debug:
+        res.out_f32 = torch.empty((T, nw.dims.embed_dim), dtype=torch.float32, device=x.device)
+        res.idx = torch.empty((T, top_k), dtype=torch.int32, device=x.device)
+        res.w = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
+        res.cnt = torch.empty((nw.dims.num_experts,), dtype=torch.int32, device=x.device)
+    p = nvfp4_params(nw, T, x, out, act_scales, top_k=top_k, router_bias=router_bias, rms_norm_out=rms_norm_out,
+                     res=res, workspace=workspace)
+    B.check(B.moe_block_forward_nvfp4(p, stream), "moe_block_forward_nvfp4")
+    return res
+
+
+def nvfp4_params(nw, T, x, out, act_scales, *, top_k=B.TOP_K, router_bias=None, rms_norm_out=False, res=None,
+                 workspace=None) -> B.MoeNvfp4Params:
+    p = B.MoeNvfp4Params()
+    p.T, p.top_k_experts = T, top_k
+    d = nw.dims
+    p.embed_dim, p.num_experts, p.expert_dim, p.hidden_dim = d.embed_dim, d.num_experts, d.expert_dim, d.hidden_dim
+    p.x, p.w_router, p.router_bias = B.ptr(x), B.ptr(nw.w_router), B.ptr(router_bias)
+    for name in ("wg", "wu", "wd", "sg", "su", "sd"):
+        setattr(p, name, getattr(nw, name).struct())
+    p.g_x, p.g_h, p.g_hs = (float(v) for v in act_scales)
+    p.rms_norm_out = 1 if rms_norm_out else 0
+    p.out = B.ptr(out)
+    if res is not None:
+        p.out_f32, p.idx_out, p.w_out, p.cnt_out = (B.ptr(res.out_f32), B.ptr(res.idx), B.ptr(res.w), B.ptr(res.cnt))
+    if workspace is not None:
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel()
+    return p
+
+
+def calibrate(dw: DeviceWeights, x: torch.Tensor, top_k: int = B.TOP_K, router_bias=None, stream=None):
+    """Static NVFP4 activation tensor scales (g_x, g_h, g_hs) = 448*6/amax from one
+    calibration batch run through the bf16 block (the library's observer)."""
+    ws, _ = workspace_for(dw.dims, x.shape[0], top_k, device=x.device)
+    out = torch.empty((x.shape[0], dw.dims.embed_dim), dtype=torch.bfloat16, device=x.device)
+    amax = torch.zeros(3, dtype=torch.float32, device=x.device)
+    p = B.make_params(x.shape[0], x, *dw.args(), out, top_k=top_k, dims=dw.dims, router_bias=router_bias, workspace=ws)
+    B.check(B.moe_nvfp4_calibrate(p, amax, stream), "moe_nvfp4_calibrate")
+    a = amax.cpu().numpy().astype(np.float32)
+    return tuple(np.float32(2688.0) / v if v > 0 else np.float32(1.0) for v in a), a

@@ -15,6 +15,7 @@
 #include "grouped_gemm.cuh"
 #include "permute.cuh"
 #include "router.cuh"
+#include "nvfp4.cuh"
 
 namespace moe {
 
@@ -139,6 +140,12 @@ moe_status device_state(DeviceState** out) {
       if (cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(fp4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(fp4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
     }
     s.init = true;
   }
@@ -219,11 +226,23 @@ enum KernelId : int {
   kKGemmDown,
   kKCombine,
   kKTimeoutProbe,
+  kKWeightAmax,
+  kKTensorScale,
+  kKWeightQuant,
+  kKActQuant,
+  kKScatterFp4,
+  kKFp4GateUp,
+  kKFp4Down,
+  kKCombineNorm,
+  kKAmax,
   kKCount
 };
 const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "build_masks", "route_scan",
                                            "route_scatter", "grouped_gemm_gateup",
-                                           "grouped_gemm_down", "combine", "timeout_probe"};
+                                           "grouped_gemm_down", "combine", "timeout_probe",
+                                           "nvfp4_weight_amax", "nvfp4_tensor_scale", "nvfp4_weight_quant",
+                                           "nvfp4_act_quant", "route_scatter_fp4", "fp4_gemm_gateup",
+                                           "fp4_gemm_down", "combine_norm", "amax"};
 
 struct ProfRecord {
   int id;
@@ -357,7 +376,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S, d.D, base, cnt, off,
                                                   reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                                   reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                                  reinterpret_cast<TileCounts*>(ws + L.counts));
+                                                  reinterpret_cast<TileCounts*>(ws + L.counts), 0);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
@@ -437,6 +456,216 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   MOE_TRY(ls_.done(le_));
   }
 
+  if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->w_out && cudaMemcpyAsync(p->w_out, w, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->cnt_out && cudaMemcpyAsync(p->cnt_out, cnt, d.E * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------- NVFP4 host
+
+// [rows, cols] bytes; box 128 bytes x 128 rows; 128-byte swizzle.
+bool map_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [groups, rows, cols] bytes; box 128 bytes x 128 rows x 1; 128-byte swizzle.
+bool map_3d_u8(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+  const cuuint64_t dims[3] = {cols, rows, groups};
+  const cuuint64_t strides[2] = {cols, rows * cols};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t fp4_q_bytes(size_t groups, size_t K, size_t N) { return groups * N * (K / 2); }
+size_t fp4_sf_bytes(size_t groups, size_t K, size_t N) { return groups * ((N + 127) / 128) * (K / 64) * 512; }
+
+// The NVFP4 workspace: the routing part (same fields as the bf16 layout) and
+// the quantised activations in a 128-padded expert-major row space.
+struct Fp4Layout {
+  Layout r;  // routing offsets (partial, idx, w, masks, base, cnt, off, row_of, tiles, counts)
+  size_t xq_perm, xsf_perm, xq_tok, xsf_tok, hq, hsf, hsq, hssf, y, s;
+  size_t total;
+  long long r_pad, t_pad;
+};
+
+Fp4Layout make_fp4_layout(const Dims& d) {
+  Fp4Layout F{};
+  Layout& L = F.r;
+  const size_t T = d.T, k = d.k, E = d.E, R = T * k;
+  L.nsplit = router_splits(d);
+  L.nchunks = static_cast<int>((T + kMaskTokens - 1) / kMaskTokens);
+  const int mt_sh = static_cast<int>((T + kBM - 1) / kBM);
+  const long long mt_max = static_cast<long long>(R / kBM) + std::min<long long>(E, R) + 1;
+  L.max_tiles_gu = static_cast<int>(((d.S + 127) / 128) * mt_sh + mt_max * ((d.F + 127) / 128));
+  L.max_tiles_dn = static_cast<int>(((d.D + 255) / 256) * mt_sh + mt_max * ((d.D + 255) / 256));
+  F.r_pad = mt_max * kBM;
+  F.t_pad = static_cast<long long>(mt_sh) * kBM;
+  const size_t rp = F.r_pad, tp = F.t_pad;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, kAlign);
+    return at;
+  };
+  L.partial = take(static_cast<size_t>(L.nsplit) * T * E * 4);
+  L.idx = take(R * 4);
+  L.w = take(R * 4);
+  L.masks = take(static_cast<size_t>(L.nchunks) * E * 4);
+  L.base = take(static_cast<size_t>(L.nchunks) * E * 4);
+  L.cnt = take(E * 4);
+  L.off = take((E + 1) * 4);
+  L.row_of = take(R * 4);
+  L.tiles_gu = take(static_cast<size_t>(L.max_tiles_gu) * sizeof(Tile));
+  L.tiles_dn = take(static_cast<size_t>(L.max_tiles_dn) * sizeof(Tile));
+  L.counts = take(sizeof(TileCounts));
+  F.xq_perm = take(rp * d.D / 2);
+  F.xsf_perm = take(rp * d.D / 16);
+  F.xq_tok = take(tp * d.D / 2);
+  F.xsf_tok = take(tp * d.D / 16);
+  F.hq = take(rp * d.F / 2);
+  F.hsf = take(rp * d.F / 16);
+  F.hsq = take(tp * d.S / 2);
+  F.hssf = take(tp * d.S / 16);
+  F.y = take(rp * d.D * 2);
+  F.s = take(T * d.D * 4);
+  F.total = o;
+  L.total = o;
+  return F;
+}
+
+Dims fp4_dims_of(const moe_nvfp4_params* p) {
+  Dims d;
+  d.T = p->T;
+  d.k = p->top_k_experts;
+  d.D = p->embed_dim ? p->embed_dim : MOE_EMBED_DIM;
+  d.E = p->num_experts ? p->num_experts : MOE_NUM_EXPERTS;
+  d.F = p->expert_dim ? p->expert_dim : MOE_EXPERT_DIM;
+  d.S = p->hidden_dim ? p->hidden_dim : MOE_HIDDEN_DIM;
+  return d;
+}
+
+bool linear_ok(const moe_nvfp4_linear& l) {
+  return l.q && l.sf && l.g && aligned16(l.q) && aligned16(l.sf) && aligned4(l.g);
+}
+
+moe_status check_fp4_args(const moe_nvfp4_params* p, Dims* d) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  *d = fp4_dims_of(p);
+  if (!dims_ok(*d) || d->D > 4096) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  if (!p->x || !p->w_router || !p->out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->out)) return MOE_ERR_ALIGNMENT;
+  const moe_nvfp4_linear* ls[] = {&p->wg, &p->wu, &p->wd, &p->sg, &p->su, &p->sd};
+  for (const moe_nvfp4_linear* l : ls)
+    if (!linear_ok(*l)) return (l->q && l->sf && l->g) ? MOE_ERR_ALIGNMENT : MOE_ERR_INVALID_ARG;
+  if (!(p->g_x > 0.f) || !(p->g_h > 0.f) || !(p->g_hs > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (p->out_f32 && !aligned16(p->out_f32)) return MOE_ERR_ALIGNMENT;
+  const void* opt4[] = {p->router_bias, p->idx_out, p->w_out, p->cnt_out};
+  for (const void* q : opt4)
+    if (q && !aligned4(q)) return MOE_ERR_ALIGNMENT;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(p->x), ob = reinterpret_cast<uintptr_t>(p->out);
+  const uintptr_t bytes = static_cast<uintptr_t>(d->T) * d->D * 2;
+  if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4Layout& F, uint8_t* ws,
+                             DeviceState* s, cudaStream_t st) {
+  const Layout& L = F.r;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  int32_t* off = reinterpret_cast<int32_t*>(ws + L.off);
+  int32_t* row_of = reinterpret_cast<int32_t*>(ws + L.row_of);
+  const uint32_t* masks = reinterpret_cast<const uint32_t*>(ws + L.masks);
+  int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
+  const TileCounts* counts = reinterpret_cast<const TileCounts*>(ws + L.counts);
+
+  MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
+  {
+    LaunchScope ls_(kKRouteScan, st);
+    const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
+                                     d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
+                                     reinterpret_cast<Tile*>(ws + L.tiles_dn),
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1);
+    MOE_TRY(ls_.done(le_));
+  }
+  {
+    const long long R = static_cast<long long>(d.T) * d.k;
+    const int blocks = static_cast<int>(std::min<long long>((R + 7) / 8, 148LL * 64));
+    LaunchScope ls_(kKScatterFp4, st);
+    const cudaError_t le_ = launch_k(route_scatter_fp4_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E,
+                                     d.D, static_cast<const __nv_bfloat16*>(p->x), p->g_x, row_of,
+                                     ws + F.xq_perm, ws + F.xsf_perm, ws + F.xq_tok, ws + F.xsf_tok);
+    MOE_TRY(ls_.done(le_));
+  }
+  const long long rp = F.r_pad, tp = F.t_pad;
+
+  Fp4Params gu;
+  std::memset(&gu, 0, sizeof(gu));
+  bool ok = map_2d_u8(&gu.tmA[0], ws + F.xq_perm, rp, d.D / 2) &&
+            map_3d_u8(&gu.tmB0[0], p->wg.q, d.E, d.F, d.D / 2) && map_3d_u8(&gu.tmB1[0], p->wu.q, d.E, d.F, d.D / 2) &&
+            map_2d_u8(&gu.tmA[1], ws + F.xq_tok, tp, d.D / 2) && map_3d_u8(&gu.tmB0[1], p->sg.q, 1, d.S, d.D / 2) &&
+            map_3d_u8(&gu.tmB1[1], p->su.q, 1, d.S, d.D / 2);
+  if (!ok) return MOE_ERR_CUDA;
+  gu.prob[0] = Fp4Problem{d.D,      d.F,      d.E,    static_cast<int>(rp), ws + F.xsf_perm, p->wg.sf, p->wu.sf,
+                          p->wg.g,  p->wu.g,  p->g_x, ws + F.hq,            ws + F.hsf,      p->g_h,   d.F / 2, 0};
+  gu.prob[1] = Fp4Problem{d.D,     d.S,     1,      static_cast<int>(tp), ws + F.xsf_tok, p->sg.sf, p->su.sf,
+                          p->sg.g, p->su.g, p->g_x, ws + F.hsq,           ws + F.hssf,    p->g_hs,  d.S / 2, 0};
+  gu.nprob = 2;
+  gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
+  gu.num_tiles = &counts->gateup;
+  gu.err = s->err;
+  {
+    LaunchScope ls_(kKFp4GateUp, st);
+    const cudaError_t le_ =
+        launch_k(fp4_gemm_kernel<true>, std::min(s->sm_count, L.max_tiles_gu), kGemmThreads, kF4SmemBytes, st, gu);
+    MOE_TRY(ls_.done(le_));
+  }
+
+  Fp4Params dn;
+  std::memset(&dn, 0, sizeof(dn));
+  ok = map_2d_u8(&dn.tmA[0], ws + F.hq, rp, d.F / 2) && map_3d_u8(&dn.tmB0[0], p->wd.q, d.E, d.D, d.F / 2) &&
+       map_2d_u8(&dn.tmA[1], ws + F.hsq, tp, d.S / 2) && map_3d_u8(&dn.tmB0[1], p->sd.q, 1, d.D, d.S / 2);
+  if (!ok) return MOE_ERR_CUDA;
+  dn.tmB1[0] = dn.tmB0[0];
+  dn.tmB1[1] = dn.tmB0[1];
+  float* sbuf = reinterpret_cast<float*>(ws + F.s);
+  dn.prob[0] = Fp4Problem{d.F,     d.D,     d.E,    static_cast<int>(rp), ws + F.hsf, p->wd.sf, p->wd.sf,
+                          p->wd.g, p->wd.g, p->g_h, ws + F.y,             nullptr,    0.f,      d.D,     0};
+  dn.prob[1] = Fp4Problem{d.S,     d.D,     1,       static_cast<int>(tp), ws + F.hssf, p->sd.sf, p->sd.sf,
+                          p->sd.g, p->sd.g, p->g_hs, sbuf,                 nullptr,     0.f,      d.D,     1};
+  dn.nprob = 2;
+  dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
+  dn.num_tiles = &counts->down;
+  dn.err = s->err;
+  {
+    LaunchScope ls_(kKFp4Down, st);
+    const cudaError_t le_ =
+        launch_k(fp4_gemm_kernel<false>, std::min(s->sm_count, L.max_tiles_dn), kGemmThreads, kF4SmemBytes, st, dn);
+    MOE_TRY(ls_.done(le_));
+  }
+  {
+    LaunchScope ls_(kKCombineNorm, st);
+    const cudaError_t le_ = launch_k(combine_norm_kernel, d.T, kCombThreads, 0, st, sbuf,
+                                     reinterpret_cast<const __nv_bfloat16*>(ws + F.y), row_of, w, d.T, d.k, d.D,
+                                     p->rms_norm_out, static_cast<__nv_bfloat16*>(p->out), p->out_f32);
+    MOE_TRY(ls_.done(le_));
+  }
+  const size_t R = static_cast<size_t>(d.T) * d.k;
   if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (p->w_out && cudaMemcpyAsync(p->w_out, w, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -717,6 +946,120 @@ moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* 
   L.partial = 0;
   L.masks = partial_bytes(L.nsplit);
   return enqueue_route(d, L, scratch, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_nvfp4_weight_bytes(int groups, int K, int N, size_t* q_bytes, size_t* sf_bytes) {
+  if (groups <= 0 || K <= 0 || N <= 0 || K % 64 || N % 64) return MOE_ERR_INVALID_ARG;
+  if (q_bytes) *q_bytes = fp4_q_bytes(groups, K, N);
+  if (sf_bytes) *sf_bytes = fp4_sf_bytes(groups, K, N);
+  return MOE_OK;
+}
+
+moe_status moe_nvfp4_quantize_weight(const void* w, int groups, int K, int N, uint8_t* q, uint8_t* sf, float* g,
+                                     void* stream) {
+  t_launches = 0;
+  if (groups <= 0 || K <= 0 || N <= 0 || K % 64 || N % 64 || groups > 65535) return MOE_ERR_INVALID_ARG;
+  if (!w || !q || !sf || !g) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(q) || !aligned16(sf) || !aligned4(g)) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(g, 0, sizeof(float) * groups, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(sf, 0, fp4_sf_bytes(groups, K, N), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t per_group = static_cast<size_t>(K) * N;
+  uint32_t* amax_bits = reinterpret_cast<uint32_t*>(g);  // amax first, then G in place
+  {
+    const int bpg = static_cast<int>(std::min<size_t>((per_group / 8 + 255) / 256, 64));
+    LaunchScope ls_(kKWeightAmax, st);
+    const cudaError_t le_ = launch_k(weight_amax_kernel, dim3(bpg, groups), 256, 0, st,
+                                     static_cast<const __nv_bfloat16*>(w), per_group, amax_bits);
+    MOE_TRY(ls_.done(le_));
+  }
+  {
+    LaunchScope ls_(kKTensorScale, st);
+    const cudaError_t le_ = launch_k(tensor_scale_kernel, (groups + 127) / 128, 128, 0, st,
+                                     static_cast<const uint32_t*>(amax_bits), g, groups);
+    MOE_TRY(ls_.done(le_));
+  }
+  const long long items = static_cast<long long>(N) * (K / 16);
+  LaunchScope ls_(kKWeightQuant, st);
+  const cudaError_t le_ = launch_k(weight_quant_kernel, dim3(static_cast<unsigned>((items + 255) / 256), groups), 256, 0,
+                                   st, static_cast<const __nv_bfloat16*>(w), K, N, static_cast<const float*>(g), q, sf);
+  return ls_.done(le_);
+}
+
+moe_status moe_nvfp4_quantize_act(const void* x, int rows, int K, float g, uint8_t* q, uint8_t* sf, void* stream) {
+  t_launches = 0;
+  if (rows < 0 || K <= 0 || K % 64 || !(g > 0.f)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !sf) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q)) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int blocks = std::min((rows + 7) / 8, s->sm_count * 16);
+  LaunchScope ls_(kKActQuant, st);
+  const cudaError_t le_ =
+      launch_k(act_quant_kernel, blocks, 256, 0, st, static_cast<const __nv_bfloat16*>(x), rows, K, g, q, sf);
+  return ls_.done(le_);
+}
+
+size_t moe_nvfp4_workspace_bytes(const moe_nvfp4_params* p) {
+  if (!p) return 0;
+  const Dims d = fp4_dims_of(p);
+  if (!dims_ok(d)) return 0;
+  return make_fp4_layout(d).total;
+}
+
+moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream) {
+  t_launches = 0;
+  Dims d;
+  MOE_TRY(check_fp4_args(p, &d));
+  if (d.T == 0) return MOE_OK;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  const Fp4Layout F = make_fp4_layout(d);
+  uint8_t* ws = nullptr;
+  if (p->workspace) {
+    if ((reinterpret_cast<uintptr_t>(p->workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGNMENT;
+    if (p->workspace_bytes < F.total) return MOE_ERR_WORKSPACE;
+    ws = static_cast<uint8_t*>(p->workspace);
+  } else {
+    void* wsv = nullptr;
+    MOE_TRY(library_workspace(s, F.total, &wsv));
+    ws = static_cast<uint8_t*>(wsv);
+  }
+  return enqueue_block_fp4(p, d, F, ws, s, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream) {
+  t_launches = 0;
+  Dims d;
+  MOE_TRY(check_block_args(p, &d));
+  if (!amax || !p->workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(amax)) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(amax, 0, 3 * sizeof(float), st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (d.T == 0) return MOE_OK;
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  const Layout L = make_layout(d);
+  uint8_t* ws = nullptr;
+  MOE_TRY(resolve_workspace(p, s, L, &ws));
+  MOE_TRY(enqueue_block(p, d, L, ws, s, st));
+  const size_t R = static_cast<size_t>(d.T) * d.k;
+  const void* srcs[3] = {p->x, ws + L.h, ws + L.hs};
+  const size_t ns[3] = {static_cast<size_t>(d.T) * d.D, R * d.F, static_cast<size_t>(d.T) * d.S};
+  for (int i = 0; i < 3; ++i) {
+    const int blocks = static_cast<int>(std::min<size_t>((ns[i] / 8 + 255) / 256, static_cast<size_t>(s->sm_count) * 8));
+    LaunchScope ls_(kKAmax, st);
+    const cudaError_t le_ = launch_k(amax_bf16_kernel, blocks, 256, 0, st, static_cast<const __nv_bfloat16*>(srcs[i]),
+                                     ns[i], reinterpret_cast<uint32_t*>(amax) + i);
+    MOE_TRY(ls_.done(le_));
+  }
+  return MOE_OK;
 }
 
 }  // extern "C"

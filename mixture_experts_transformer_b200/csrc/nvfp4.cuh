@@ -1,0 +1,661 @@
+// NVFP4 variant of the block: e2m1 values in groups of 16 along K with e4m3
+// group scales and an fp32 tensor scale (G4-MeroMero-26B-A4B-NVFP4
+// config.json, quantization_config.config_groups.group_0: "num_bits": 4,
+// "type": float, "group_size": 16, "scale_dtype": float8_e4m3fn, strategy
+// "tensor_group"; weights static, input activations "dynamic": "local"; the
+// routers stay bf16, they are on the "ignore" list).
+//
+// Quantisation, per group of 16 values under tensor scale G (all fp32, IEEE
+// round-to-nearest operations, so the codes are reproducible bit for bit):
+//   G     = 448 * 6 / amax(tensor)                  (weights; activations: calibrated)
+//   s     = e4m3_satfinite(RN(RN(amax16 / 6) * G))  (s = 0: the whole group is 0)
+//   q_i   = e2m1_satfinite(RN(x_i * RN(G / s)))
+//   x^_i  = e2m1(q_i) * s / G
+//
+// Storage (also the tcgen05 block-scaled operand layout):
+//   codes  [rows][K/2] bytes, K-major, element 2j in the low nibble of byte j;
+//   scales [rows/128][K/64][512] bytes: the 16-bit-group scales of rows
+//          128a .. 128a+127 and K range 64b .. 64b+63 form one 512-byte atom,
+//          row r, group c (0..3) at byte 16*(r%32) + 4*(r/32) + c.
+//
+// The GEMM (fp4_gemm_kernel) is the bf16 grouped GEMM's structure with
+// `tcgen05.mma.kind::mxf4nvf4.block_scale.block16`: TMA brings 256-K stages of
+// A and B codes plus the matching scale atoms (a bulk copy), the MMA thread
+// moves each 64-K step's scale atoms into TMEM with tcgen05.cp (32x128b,
+// broadcast to the four lane quarters) and issues two M=128, N=128 MMAs.
+// The epilogue multiplies by 1/(G_act * G_weight); the gate|up epilogue then
+// quantises the GeGLU rows h to NVFP4 for the down projection.
+#pragma once
+
+#include "grouped_gemm.cuh"
+#include "ptx.cuh"
+#include "router.cuh"
+
+namespace moe {
+
+constexpr float kFp4Max = 6.0f;
+constexpr float kE4m3Max = 448.0f;
+
+// ----------------------------------------------------------- quantisation
+
+__device__ __forceinline__ uint32_t e4m3_code(float v) {  // v >= 0, finite
+  unsigned short s;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(s) : "f"(0.0f), "f"(v));
+  return s & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t c) {  // c in [0, 0x7E]
+  const uint32_t e = (c >> 3) & 0xFu, m = c & 7u;
+  if (e == 0) return static_cast<float>(m) * 0.001953125f;  // m * 2^-9
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));    // (1 + m/8) * 2^(e-7)
+}
+
+// two e2m1 codes in one byte: lo in bits 0-3, hi in bits 4-7
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Quantise 16 values under tensor scale g: returns the scale code, writes the
+// 8 code bytes (little-endian: value 0 in the low nibble of byte 0) to *codes.
+__device__ __forceinline__ uint32_t nvfp4_group(const float (&v)[16], float g, uint2* codes) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sc = e4m3_code(__fmul_rn(__fdiv_rn(amax, kFp4Max), g));
+  const float sv = e4m3_value(sc);
+  uint32_t w[2] = {0u, 0u};
+  if (sv > 0.f) {
+    const float r = __fdiv_rn(g, sv);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int i = h * 8 + b * 2;
+        word |= e2m1x2(__fmul_rn(v[i], r), __fmul_rn(v[i + 1], r)) << (8 * b);
+      }
+      w[h] = word;
+    }
+  }
+  *codes = make_uint2(w[0], w[1]);
+  return sc;
+}
+
+// Byte offset of the scale of (row, group c16) in a [rows/128][K/64][512] atom array.
+__device__ __forceinline__ size_t sf_offset(int row, int c16, int k64_blocks) {
+  return (static_cast<size_t>(row >> 7) * k64_blocks + (c16 >> 2)) * 512 + 16 * (row & 31) + 4 * ((row & 127) >> 5) +
+         (c16 & 3);
+}
+
+__device__ __forceinline__ void load16_bf16(const __nv_bfloat16* p, float (&v)[16]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  const __nv_bfloat16* pa = reinterpret_cast<const __nv_bfloat16*>(&a);
+  const __nv_bfloat16* pb = reinterpret_cast<const __nv_bfloat16*>(&b);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = __bfloat162float(pa[i]);
+    v[8 + i] = __bfloat162float(pb[i]);
+  }
+}
+
+// ------------------------------------------------------- weight quantiser
+
+// amax over each group's [K][N] matrix into amax_bits[g] (float bits; amax >= 0
+// so the integer maximum is the float maximum). amax_bits must be zero.
+__global__ void weight_amax_kernel(const __nv_bfloat16* __restrict__ w, size_t per_group,
+                                   uint32_t* __restrict__ amax_bits) {
+  pdl_wait_then_release();
+  const int g = blockIdx.y;
+  const __nv_bfloat16* base = w + per_group * g;
+  float m = 0.f;
+  for (size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < per_group;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x * 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + i));
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(__bfloat162float(b[j])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits + g, __float_as_uint(m));
+}
+
+// G = 448 * 6 / amax (1 for an all-zero tensor).
+__global__ void tensor_scale_kernel(const uint32_t* __restrict__ amax_bits, float* __restrict__ g, int n) {
+  pdl_wait_then_release();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float a = __uint_as_float(amax_bits[i]);
+  g[i] = a > 0.f ? __fdiv_rn(kE4m3Max * kFp4Max, a) : 1.0f;
+}
+
+// One thread per (n, 16-group of K) of w [G][K][N] (N contiguous): codes into
+// q [G][N][K/2], scale into the atoms of sf [G][ceil(N/128)][K/64][512]
+// (cleared beforehand, so padding rows keep scale 0).
+__global__ void weight_quant_kernel(const __nv_bfloat16* __restrict__ w, int K, int N, const float* __restrict__ gs,
+                                    uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  pdl_wait_then_release();
+  const int g = blockIdx.y;
+  const int kg_count = K / 16;
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(N) * kg_count) return;
+  const int n = static_cast<int>(idx % N);
+  const int kg = static_cast<int>(idx / N);
+  const __nv_bfloat16* src = w + (static_cast<size_t>(g) * K + kg * 16) * N + n;
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __bfloat162float(src[static_cast<size_t>(i) * N]);
+  uint2 codes;
+  const uint32_t sc = nvfp4_group(v, gs[g], &codes);
+  *reinterpret_cast<uint2*>(q + (static_cast<size_t>(g) * N + n) * (K / 2) + kg * 8) = codes;
+  const int nb = (N + 127) / 128;
+  sf[static_cast<size_t>(g) * nb * (K / 64) * 512 + sf_offset(n, kg, K / 64)] = static_cast<uint8_t>(sc);
+}
+
+// --------------------------------------------------- activation quantiser
+
+// One warp per row of x [rows][K] bf16 -> q [rows][K/2] and the row's scales.
+__global__ void act_quant_kernel(const __nv_bfloat16* __restrict__ x, int rows, int K, float g,
+                                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  pdl_wait_then_release();
+  const int lane = threadIdx.x & 31;
+  for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += gridDim.x * 8) {
+    for (int c = lane; c < K / 16; c += 32) {
+      float v[16];
+      load16_bf16(x + static_cast<size_t>(r) * K + c * 16, v);
+      uint2 codes;
+      const uint32_t sc = nvfp4_group(v, g, &codes);
+      *reinterpret_cast<uint2*>(q + static_cast<size_t>(r) * (K / 2) + c * 8) = codes;
+      sf[sf_offset(r, c, K / 64)] = static_cast<uint8_t>(sc);
+    }
+  }
+}
+
+// The NVFP4 block's scatter: one warp per (token, slot); its routed row in the
+// 128-padded expert-major row space comes from the bitmasks, the warp
+// quantises x[t] into that row (codes + scales) and, for slot 0, also into the
+// token-order buffer the shared MLP reads.
+__global__ void __launch_bounds__(256) route_scatter_fp4_kernel(
+    const int32_t* __restrict__ idx, const uint32_t* __restrict__ masks, const int32_t* __restrict__ base, int T,
+    int k, int E, int D, const __nv_bfloat16* __restrict__ x, float g_x, int32_t* __restrict__ row_of,
+    uint8_t* __restrict__ xq_perm, uint8_t* __restrict__ xsf_perm, uint8_t* __restrict__ xq_tok,
+    uint8_t* __restrict__ xsf_tok) {
+  pdl_wait_then_release();
+  const int lane = threadIdx.x & 31;
+  const long long R = static_cast<long long>(T) * k;
+  for (long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); a < R;
+       a += static_cast<long long>(gridDim.x) * 8) {
+    const int t = static_cast<int>(a / k);
+    const int j = static_cast<int>(a % k);
+    const int e = __ldg(idx + a);
+    if (e < 0 || e >= E) continue;
+    const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
+    const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
+    const int row = __ldg(base + cw) + __popc(below);
+    if (lane == 0) row_of[a] = row;
+    for (int c = lane; c < D / 16; c += 32) {
+      float v[16];
+      load16_bf16(x + static_cast<size_t>(t) * D + c * 16, v);
+      uint2 codes;
+      const uint32_t sc = nvfp4_group(v, g_x, &codes);
+      *reinterpret_cast<uint2*>(xq_perm + static_cast<size_t>(row) * (D / 2) + c * 8) = codes;
+      xsf_perm[sf_offset(row, c, D / 64)] = static_cast<uint8_t>(sc);
+      if (j == 0) {
+        *reinterpret_cast<uint2*>(xq_tok + static_cast<size_t>(t) * (D / 2) + c * 8) = codes;
+        xsf_tok[sf_offset(t, c, D / 64)] = static_cast<uint8_t>(sc);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- FP4 GEMM
+
+constexpr int kF4KStage = 256;                   // K elements per stage (128 bytes of codes per row)
+constexpr int kF4ABytes = 128 * 128;             // 128 rows x 128 B
+constexpr int kF4BBytes = 2 * 128 * 128;         // two 128-row blocks
+constexpr int kF4SfBytes = 4 * 512;              // 4 atoms (4 x 64 K) of one 128-row block
+constexpr int kF4Stages = 4;
+constexpr int kF4SfSlots = 16;                   // TMEM scale slots (ring over 64-K steps)
+constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 1024 + 256;
+
+struct Fp4Problem {
+  int K;          // multiple of 64
+  int N;          // multiple of 64
+  int groups;
+  int a_rows;     // rows of A (a multiple of 128)
+  const uint8_t* sfa;   // [a_rows/128][K/64][512]
+  const uint8_t* sfb0;  // [groups][ceil(N/128)][K/64][512]
+  const uint8_t* sfb1;  // (up; GATEUP only)
+  const float* gb0;     // [groups] weight tensor scales
+  const float* gb1;
+  float ga;             // activation tensor scale
+  void* out;            // GATEUP: codes [rows][N/2]; DOWN: bf16 / fp32 [rows][ldo]
+  uint8_t* out_sf;      // GATEUP: scales [rows/128][N/64][512]
+  float g_out;          // GATEUP: tensor scale of the quantised output
+  int ldo;
+  int out_f32;
+};
+
+struct Fp4Params {
+  CUtensorMap tmA[2];   // codes [a_rows][K/2] u8, box 128 x 128, 128-byte swizzle
+  CUtensorMap tmB0[2];  // codes [groups][N][K/2] u8, box 128 x 128 x 1
+  CUtensorMap tmB1[2];
+  Fp4Problem prob[2];
+  int nprob;
+  const Tile* tiles;
+  const int32_t* num_tiles;
+  uint32_t* err;
+};
+
+// Instruction descriptor of kind::mxf4nvf4 (e2m1 A and B, ue4m3 scales),
+// K-major A and B, M = 128.
+__host__ __device__ constexpr uint32_t idesc_nvf4_m128(int n) {
+  return (1u << 7)                                  // A format e2m1
+         | (1u << 10)                               // B format e2m1
+         | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(128 >> 4) << 24);   // M / 16
+}
+
+// Shared-memory descriptor of one 512-byte scale atom for tcgen05.cp
+// (no swizzle, K-major: 8-row groups of 16-byte rows, 128 bytes apart).
+__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128 >> 4) << 32;  // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+template <bool GATEUP>
+__device__ __forceinline__ int f4_tile_cols(const Fp4Problem& pr, int n0) {
+  const int cap = GATEUP ? 128 : 256;
+  const int rem = pr.N - n0;
+  return rem < cap ? rem : cap;
+}
+
+// TMEM columns: accumulator [0, 256) (GATEUP: gate 0..127, up 128..255; DOWN:
+// output columns n0 .. n0+255), scale slots from 256: slot i holds the A
+// scales at +0, B block 0 at +4, B block 1 at +8.
+template <bool GATEUP>
+__global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_constant__ Fp4Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + kF4Stages * kF4ABytes;
+  uint8_t* sSfA = sB + kF4Stages * kF4BBytes;
+  uint8_t* sSfB = sSfA + kF4Stages * kF4SfBytes;  // per stage: block 0 atoms, then block 1 atoms
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + kF4Stages * 2 * kF4SfBytes);
+  uint64_t* empty = full + kF4Stages;
+  uint64_t* acc_full = empty + kF4Stages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kF4Stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int p = 0; p < P.nprob; ++p) {
+      tma_prefetch_desc(&P.tmA[p]);
+      tma_prefetch_desc(&P.tmB0[p]);
+      tma_prefetch_desc(&P.tmB1[p]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_then_release();
+  const int num_tiles = *P.num_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+        const Tile tile = P.tiles[ti];
+        const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+        if (p >= P.nprob) {
+          atomicOr(P.err, kErrBadTile);
+          *abort_flag = 1;
+          break;
+        }
+        const Fp4Problem& pr = P.prob[p];
+        if (g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || (tile.row0 & 127) || tile.n0 < 0 ||
+            tile.n0 >= pr.N) {
+          atomicOr(P.err, kErrBadTile);
+          *abort_flag = 1;
+          break;
+        }
+        const int k64 = pr.K / 64;
+        const int nstage = (pr.K + kF4KStage - 1) / kF4KStage;
+        const int nbr = (pr.N + 127) / 128;
+        const int nb0 = tile.n0 >> 7;
+        const int nb1 = GATEUP ? nb0 : nb0 + 1;
+        const uint8_t* sfa = pr.sfa + static_cast<size_t>(tile.row0 >> 7) * k64 * 512;
+        const uint8_t* sfb0 = pr.sfb0 + (static_cast<size_t>(g) * nbr + nb0) * k64 * 512;
+        const uint8_t* sfb1 = (GATEUP ? pr.sfb1 : pr.sfb0) + (static_cast<size_t>(g) * nbr + nb1) * k64 * 512;
+        const bool two_b = GATEUP || (tile.n0 + 128 < pr.N);
+        bool ok = true;
+        for (int ks = 0; ks < nstage; ++ks) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          const int nks = min(4, k64 - 4 * ks);
+          const uint32_t sf_bytes = nks * 512;
+          const uint32_t bytes = kF4ABytes + (two_b ? 2 : 1) * (kF4BBytes / 2) + sf_bytes * (two_b ? 3 : 2);
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d(sA + s * kF4ABytes, &P.tmA[p], &full[s], ks * 128, tile.row0);
+          tma_load_3d(sB + s * kF4BBytes, &P.tmB0[p], &full[s], ks * 128, tile.n0, g);
+          if (two_b) {
+            if (GATEUP)
+              tma_load_3d(sB + s * kF4BBytes + kF4BBytes / 2, &P.tmB1[p], &full[s], ks * 128, tile.n0, g);
+            else
+              tma_load_3d(sB + s * kF4BBytes + kF4BBytes / 2, &P.tmB0[p], &full[s], ks * 128, tile.n0 + 128, g);
+          }
+          bulk_load(sSfA + s * kF4SfBytes, sfa + static_cast<size_t>(4 * ks) * 512, sf_bytes, &full[s]);
+          bulk_load(sSfB + (2 * s) * kF4SfBytes, sfb0 + static_cast<size_t>(4 * ks) * 512, sf_bytes, &full[s]);
+          if (two_b)
+            bulk_load(sSfB + (2 * s + 1) * kF4SfBytes, sfb1 + static_cast<size_t>(4 * ks) * 512, sf_bytes, &full[s]);
+          ++issued;
+          if (++s == kF4Stages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        int st = s;
+        uint32_t sp = ph;
+        const int pending = issued < kF4Stages ? issued : kF4Stages;
+        for (int i = 0; i < pending; ++i) {
+          if (--st < 0) {
+            st = kF4Stages - 1;
+            sp ^= 1;
+          }
+          uint32_t dummy = 0;
+          mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      int s = 0, slot = 0;
+      uint32_t ph = 0, acc_ph = 0;
+      bool any = false;
+      const uint32_t idesc = idesc_nvf4_m128(128);
+      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+        const Tile tile = P.tiles[ti];
+        const int p = tile.pg >> 16;
+        if (p >= P.nprob) break;
+        const Fp4Problem& pr = P.prob[p];
+        const int k64 = pr.K / 64;
+        const int nstage = (pr.K + kF4KStage - 1) / kF4KStage;
+        const bool two_b = GATEUP || (tile.n0 + 128 < pr.N);
+        if (!mbar_wait(acc_empty, acc_ph ^ 1, abort_flag, P.err)) break;
+        tc_fence_after_sync();
+        bool ok = true;
+        for (int ks = 0; ks < nstage; ++ks) {
+          if (!mbar_wait(&full[s], ph, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const int nks = min(4, k64 - 4 * ks);
+          const uint32_t a_addr = smem_u32(sA + s * kF4ABytes);
+          const uint32_t b_addr = smem_u32(sB + s * kF4BBytes);
+          const uint32_t sfa_addr = smem_u32(sSfA + s * kF4SfBytes);
+          const uint32_t sfb_addr = smem_u32(sSfB + (2 * s) * kF4SfBytes);
+          for (int i = 0; i < nks; ++i) {
+            const uint32_t cols = tmem_base + kAccCols + slot * 16;
+            tmem_cp_32x128b_x4(cols, sdesc_sf_atom(sfa_addr + i * 512));
+            tmem_cp_32x128b_x4(cols + 4, sdesc_sf_atom(sfb_addr + i * 512));
+            if (two_b) tmem_cp_32x128b_x4(cols + 8, sdesc_sf_atom(sfb_addr + kF4SfBytes + i * 512));
+            // 64 K of e2m1 = 32 B per row inside the 128-byte swizzled rows
+            const uint64_t ad = sdesc_sw128(a_addr + i * 32, 16, 1024);
+            const uint64_t bd0 = sdesc_sw128(b_addr + i * 32, 16, 1024);
+            const uint32_t acc = (ks | i) != 0;
+            umma_nvf4(tmem_base, ad, bd0, idesc, cols, cols + 4, acc);
+            if (two_b) {
+              const uint64_t bd1 = sdesc_sw128(b_addr + kF4BBytes / 2 + i * 32, 16, 1024);
+              umma_nvf4(tmem_base + 128, ad, bd1, idesc, cols, cols + 8, acc);
+            }
+            slot = (slot + 1) % kF4SfSlots;
+          }
+          any = true;
+          umma_commit(&empty[s]);
+          if (++s == kF4Stages) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(acc_full);
+        acc_ph ^= 1;
+      }
+      if (any) {
+        umma_commit(drain);
+        uint32_t dummy = 0;
+        mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), P.err);
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    uint32_t acc_ph = 0;
+    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      const Tile tile = P.tiles[ti];
+      const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+      if (p >= P.nprob) break;
+      const Fp4Problem& pr = P.prob[p];
+      const int wn = f4_tile_cols<GATEUP>(pr, tile.n0);
+      const bool ready = mbar_wait(acc_full, acc_ph, abort_flag, P.err);
+      __syncwarp();
+      if (!ready) break;
+      tc_fence_after_sync();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      const bool valid = r < tile.rows;
+      const int grow = tile.row0 + r;
+      if (GATEUP) {
+        const float ag = 1.0f / (pr.ga * pr.gb0[g]);
+        const float au = 1.0f / (pr.ga * pr.gb1[g]);
+        uint8_t* q = reinterpret_cast<uint8_t*>(pr.out) + static_cast<size_t>(grow) * (pr.N / 2);
+        for (int j = 0; j < wn; j += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld_32x32b_x32(tbase + j, gv);
+          tmem_ld_32x32b_x32(tbase + 128 + j, uv);
+          tmem_ld_wait();
+          uint2 codes[2];
+          uint32_t sc[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              v[i] = gelu_tanh(__uint_as_float(gv[16 * h + i]) * ag) * (__uint_as_float(uv[16 * h + i]) * au);
+            sc[h] = nvfp4_group(v, pr.g_out, &codes[h]);
+          }
+          if (valid) {
+            *reinterpret_cast<uint4*>(q + (tile.n0 + j) / 2) = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+            const int c16 = (tile.n0 + j) / 16;
+            pr.out_sf[sf_offset(grow, c16, pr.N / 64)] = static_cast<uint8_t>(sc[0]);
+            pr.out_sf[sf_offset(grow, c16 + 1, pr.N / 64)] = static_cast<uint8_t>(sc[1]);
+          }
+        }
+      } else {
+        const float alpha = 1.0f / (pr.ga * pr.gb0[g]);
+        for (int j = 0; j < wn; j += 32) {
+          uint32_t a[32];
+          tmem_ld_32x32b_x32(tbase + j, a);
+          tmem_ld_wait();
+          if (valid) {
+            if (pr.out_f32) {
+              float4* dst =
+                  reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(a[4 * v]) * alpha, __uint_as_float(a[4 * v + 1]) * alpha,
+                                     __uint_as_float(a[4 * v + 2]) * alpha, __uint_as_float(a[4 * v + 3]) * alpha);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) +
+                                                    static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(
+                    pack_bf16x2(__uint_as_float(a[8 * v]) * alpha, __uint_as_float(a[8 * v + 1]) * alpha),
+                    pack_bf16x2(__uint_as_float(a[8 * v + 2]) * alpha, __uint_as_float(a[8 * v + 3]) * alpha),
+                    pack_bf16x2(__uint_as_float(a[8 * v + 4]) * alpha, __uint_as_float(a[8 * v + 5]) * alpha),
+                    pack_bf16x2(__uint_as_float(a[8 * v + 6]) * alpha, __uint_as_float(a[8 * v + 7]) * alpha));
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      acc_ph ^= 1;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------- combine
+
+// out[t] = s[t] + sum_j w[t, j] y[row_of[t, j]] in fp32 (slot order), then
+// optionally x / sqrt(mean(x^2) + 1e-6) (the unlearned RMSNorm between the
+// blocks of the NVFP4 stack; model card: RMSNorm, eps 1e-06). One CTA per
+// token; each thread keeps up to kCombVec 8-column vectors in registers.
+constexpr int kCombThreads = 128;
+constexpr int kCombVec = 4;  // supports D <= 128 * 4 * 8 = 4096
+
+__global__ void __launch_bounds__(kCombThreads) combine_norm_kernel(
+    const float* __restrict__ s, const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ row_of,
+    const float* __restrict__ w, int T, int k, int D, int rms_norm, __nv_bfloat16* __restrict__ out,
+    float* __restrict__ out_f32) {
+  __shared__ int s_row[128];
+  __shared__ float s_w[128];
+  __shared__ float s_red[kCombThreads / 32];
+  pdl_wait_then_release();
+  const int t = blockIdx.x;
+  for (int j = threadIdx.x; j < k; j += blockDim.x) {
+    s_row[j] = row_of[static_cast<size_t>(t) * k + j];
+    s_w[j] = w[static_cast<size_t>(t) * k + j];
+  }
+  __syncthreads();
+  const int nvec = D >> 3;
+  float acc[kCombVec][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < kCombVec; ++u) {
+    const int v = threadIdx.x + u * kCombThreads;
+    if (v >= nvec) continue;
+    const float4* sp = reinterpret_cast<const float4*>(s + static_cast<size_t>(t) * D) + 2 * v;
+    const float4 s0 = sp[0], s1 = sp[1];
+    acc[u][0] = s0.x; acc[u][1] = s0.y; acc[u][2] = s0.z; acc[u][3] = s0.w;
+    acc[u][4] = s1.x; acc[u][5] = s1.y; acc[u][6] = s1.z; acc[u][7] = s1.w;
+    for (int j = 0; j < k; ++j) {
+      const uint4 yv = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(s_row[j]) * D) + v);
+      const __nv_bfloat16* yb = reinterpret_cast<const __nv_bfloat16*>(&yv);
+      const float wj = s_w[j];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[u][i] = fmaf(wj, __bfloat162float(yb[i]), acc[u][i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(acc[u][i], acc[u][i], ss);
+  }
+  float scale = 1.0f;
+  if (rms_norm) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    for (int i = 0; i < kCombThreads / 32; ++i) tot += s_red[i];
+    scale = 1.0f / sqrtf(tot / static_cast<float>(D) + 1e-6f);
+  }
+#pragma unroll
+  for (int u = 0; u < kCombVec; ++u) {
+    const int v = threadIdx.x + u * kCombThreads;
+    if (v >= nvec) continue;
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = acc[u][i] * scale;
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * D)[v] =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+    if (out_f32) {
+      float4* op = reinterpret_cast<float4*>(out_f32 + static_cast<size_t>(t) * D) + 2 * v;
+      op[0] = make_float4(o[0], o[1], o[2], o[3]);
+      op[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+// amax of |a| over n fp32 / bf16 values into *amax_bits (zero on entry).
+__global__ void amax_bf16_kernel(const __nv_bfloat16* __restrict__ a, size_t n, uint32_t* __restrict__ amax_bits) {
+  pdl_wait_then_release();
+  float m = 0.f;
+  for (size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x * 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(a + i));
+    const __nv_bfloat16* b = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(__bfloat162float(b[j])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+}  // namespace moe

@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
                                                                   int32_t* __restrict__ off_out,
                                                                   Tile* __restrict__ tiles_gu,
                                                                   Tile* __restrict__ tiles_dn,
-                                                                  TileCounts* __restrict__ counts) {
+                                                                  TileCounts* __restrict__ counts, int padded) {
   __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
@@ -109,8 +109,11 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   }
   __syncthreads();
   const int c_e = s_cnt[e];
+  // first routed row of expert e: packed (bf16 path) or padded to whole
+  // 128-row tiles (NVFP4 path: every tile starts on a scale-atom boundary)
+  const int row_base = padded ? s_mtoff[e] * kBM : s_off[e];
   if (e < E) {
-    int run = s_off[e] + s_seg[seg][e];
+    int run = row_base + s_seg[seg][e];
     for (int c = c0; c < c1; ++c) {
       base[static_cast<size_t>(c) * E + e] = run;
       run += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
@@ -142,11 +145,11 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     const int base_dn = n_sh_dn + s_mtoff[e] * nt_dn;
     for (int i = seg; i < nt_gu * mt; i += kScanSegs) {
       const int nt = i / mt, m = i % mt;
-      tiles_gu[base_gu + i] = Tile{e, s_off[e] + m * kBM, min(kBM, c_e - m * kBM), nt * 128};
+      tiles_gu[base_gu + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * 128};
     }
     for (int i = seg; i < nt_dn * mt; i += kScanSegs) {
       const int nt = i / mt, m = i % mt;
-      tiles_dn[base_dn + i] = Tile{e, s_off[e] + m * kBM, min(kBM, c_e - m * kBM), nt * 256};
+      tiles_dn[base_dn + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * 256};
     }
   }
   if (threadIdx.x == 0) {

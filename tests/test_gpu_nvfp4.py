@@ -1,0 +1,152 @@
+"""NVFP4 path on a B200 against the oracle: quantisers bit-exact, block within
+5e-2 * RMS of the oracle's NVFP4 block (own dequantised weights, same
+activation scales, the GPU's routing)."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import SMALL, check_routing, device_weights, require_gpu, to_np, w_args, weights
+from mixture_experts_transformer_b200 import binding as B
+from mixture_experts_transformer_b200 import block, inputs
+from oracle import moe_oracle as mo
+from oracle import nvfp4 as nv
+
+pytestmark = pytest.mark.gpu
+NVFP4_TOL = 5e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def decode_layout(q_bytes: np.ndarray, sf_bytes: np.ndarray, G: int, K: int, N: int):
+    """The library's storage -> (codes [G][N][K], scale codes [G][N][K/16])."""
+    q = q_bytes.reshape(G, N, K // 2)
+    codes = np.empty((G, N, K), np.uint8)
+    codes[..., 0::2] = q & 0xF
+    codes[..., 1::2] = q >> 4
+    nb = (N + 127) // 128
+    atoms = sf_bytes.reshape(G, nb, K // 64, 512)
+    n = np.arange(N)[:, None]
+    c = np.arange(K // 16)[None, :]
+    off = 16 * (n % 32) + 4 * ((n % 128) // 32) + (c % 4)
+    scales = atoms[:, n // 128, c // 4, off]
+    return codes, scales
+
+
+def same_codes(got, ref):
+    """Equal codes, except that +0 and -0 (codes 0 and 8) count as the same value."""
+    g = np.where(got == 8, 0, got)
+    r = np.where(ref == 8, 0, ref)
+    return np.array_equal(g, r)
+
+
+@pytest.mark.parametrize("G,K,N", [(3, 256, 192), (2, 704, 128), (1, 128, 320)])
+def test_weight_quantizer_bit_exact(G, K, N):
+    rng = np.random.default_rng(G * K + N)
+    w32 = (rng.standard_normal((G, K, N)) * np.exp(rng.uniform(-4, 2, (G, 1, N)))).astype(np.float32)
+    w32[0, :16, 3] = 0.0  # an all-zero group
+    wb = inputs.f32_to_bf16_bits(w32)
+    lin = block.quantize_linear(block.bf16_tensor(wb))
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status() == B.MOE_OK
+    codes, scales = decode_layout(to_np(lin.q), to_np(lin.sf), G, K, N)
+    gs = to_np(lin.g)
+    for g in range(G):
+        wt = inputs.bf16_bits_to_f32(wb[g]).T  # [N][K]
+        G_ref = nv.tensor_scale(np.abs(wt).max())
+        assert gs[g] == G_ref
+        q_ref, s_ref = nv.quantize(wt, G_ref)
+        np.testing.assert_array_equal(scales[g], s_ref)
+        assert same_codes(codes[g], q_ref)
+    # scale rows past N are zero
+    nb = (N + 127) // 128
+    if N % 128:
+        atoms = to_np(lin.sf).reshape(G, nb, K // 64, 512)
+        pad_rows = np.arange(N % 128, 128)
+        offs = (16 * (pad_rows % 32) + 4 * (pad_rows // 32))[:, None] + np.arange(4)[None, :]
+        assert not atoms[:, nb - 1][:, :, offs.ravel()].any()
+
+
+def test_activation_quantizer_bit_exact():
+    rows, K = 300, 512
+    x = inputs.make_x(rows, K, seed=12)
+    g = np.float32(2688.0 / 4.5)  # a static scale below the data's amax: some values saturate
+    q = torch.empty(rows * K // 2, dtype=torch.uint8, device="cuda")
+    sf = torch.zeros(((rows + 127) // 128) * 128 * K // 16, dtype=torch.uint8, device="cuda")
+    B.check(B.moe_nvfp4_quantize_act(block.bf16_tensor(x), rows, K, g, q, sf), "quantize_act")
+    rpad = (rows + 127) // 128 * 128
+    codes, scales = decode_layout(
+        np.concatenate([to_np(q), np.zeros((rpad - rows) * K // 2, np.uint8)]), to_np(sf), 1, K, rpad
+    )
+    q_ref, s_ref = nv.quantize(inputs.bf16_bits_to_f32(x), g)
+    np.testing.assert_array_equal(scales[0, :rows], s_ref)
+    assert same_codes(codes[0, :rows], q_ref)
+
+
+def test_calibration_observer():
+    T = 96
+    w = weights(SMALL, seed=1, std=0.05)
+    dw = device_weights(SMALL, seed=1, std=0.05)
+    x_bits = inputs.make_x(T, SMALL.embed_dim, seed=2)
+    (gx, gh, ghs), amax = block.calibrate(dw, block.bf16_tensor(x_bits), top_k=4)
+    ref = nv.act_scales_from_calibration(x_bits, *w_args(w), top_k=4)
+    assert gx == ref[0]  # x is exact bf16 on both sides
+    # the GPU observes the bf16-stored hidden rows: within one bf16 rounding
+    np.testing.assert_allclose([gh, ghs], ref[1:], rtol=2.0**-7)
+
+
+def _oracle_block(w, x_bits, scales, routing):
+    return nv.moe_block_nvfp4(x_bits, *w_args(w), *scales, routing=routing)["out"]
+
+
+@pytest.mark.parametrize("T,k", [(1, 4), (70, 4), (300, 8)])
+def test_nvfp4_block_small_dims(T, k):
+    w = weights(SMALL, seed=1, std=0.05)
+    dw = device_weights(SMALL, seed=1, std=0.05)
+    nw = block.quantize_block(dw)
+    scales = nv.act_scales_from_calibration(inputs.make_x(64, SMALL.embed_dim, seed=2), *w_args(w), top_k=k)
+    x_bits = inputs.make_x(T, SMALL.embed_dim, seed=20 + T)
+    res = block.forward_nvfp4(nw, block.bf16_tensor(x_bits), scales, top_k=k, debug=True)
+    assert B.moe_get_device_status() == B.MOE_OK
+    idx, wts = to_np(res.idx), to_np(res.w)
+    ref_idx, ref_w, logits = mo.route(x_bits, w.w_router, k)
+    check_routing(logits, ref_idx, ref_w, idx, wts, k)  # the router stays bf16
+    ref = _oracle_block(w, x_bits, scales, (idx, wts))
+    rms = np.sqrt(np.mean(ref**2))
+    err = np.abs(to_np(res.out_f32) - ref).max()
+    assert err <= NVFP4_TOL * rms, (err / rms)
+    out_bits = res.out.float().cpu().numpy()
+    rne = torch.from_numpy(to_np(res.out_f32)).to(torch.bfloat16).float().numpy()
+    np.testing.assert_array_equal(out_bits, rne)
+
+
+def test_nvfp4_block_gemma_T64():
+    T = 64
+    w = weights()
+    dw = device_weights()
+    nw = block.quantize_block(dw)
+    scales = nv.act_scales_from_calibration(inputs.make_x(64, seed=2), *w_args(w))
+    x_bits = inputs.make_x(T)
+    res = block.forward_nvfp4(nw, block.bf16_tensor(x_bits), scales, debug=True)
+    assert B.moe_get_device_status() == B.MOE_OK
+    idx, wts = to_np(res.idx), to_np(res.w)
+    ref = _oracle_block(w, x_bits, scales, (idx, wts))
+    rms = np.sqrt(np.mean(ref**2))
+    err = np.abs(to_np(res.out_f32) - ref).max()
+    assert err <= NVFP4_TOL * rms, (err / rms)
+
+
+def test_nvfp4_rms_norm_output():
+    T = 40
+    w = weights(SMALL, seed=1, std=0.05)
+    dw = device_weights(SMALL, seed=1, std=0.05)
+    nw = block.quantize_block(dw)
+    scales = nv.act_scales_from_calibration(inputs.make_x(64, SMALL.embed_dim, seed=2), *w_args(w), top_k=4)
+    x = block.bf16_tensor(inputs.make_x(T, SMALL.embed_dim, seed=5))
+    plain = block.forward_nvfp4(nw, x, scales, top_k=4, debug=True)
+    normed = block.forward_nvfp4(nw, x, scales, top_k=4, debug=True, rms_norm_out=True)
+    ref = mo.rms_normalize(to_np(plain.out_f32))
+    np.testing.assert_allclose(to_np(normed.out_f32), ref, rtol=1e-5, atol=1e-6)
