@@ -47,7 +47,15 @@ WORKLOADS = {
     "skewed": dict(
         T=16384, bias=True, bound="tensor", desc="Gemma-4-26B-A4B MoE block, T=16384, Zipf(1.1) router bias, bf16"
     ),
+    "nvfp4_stack": dict(
+        T=2048,
+        bias=False,
+        bound="hbm",
+        layers=30,
+        desc="30 Gemma-4-26B-A4B MoE blocks in NVFP4 (group 16, e4m3 scales), RMSNorm between blocks, T=2048",
+    ),
 }
+FP4_TFLOPS_NOMINAL_RATIO = 4.0  # dense fp4 : bf16 tensor throughput, nominal (9 : 2.25 PFLOP/s)
 METRIC = "MoE-block tokens/s"
 
 NVML_REASONS = {
@@ -70,6 +78,7 @@ def parse():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None, help="nvfp4_stack depth (default 30)")
     return ap.parse_args()
 
 
@@ -426,6 +435,204 @@ def run_ours(args, world, rank, local):
     return res
 
 
+# ------------------------------------------------------------ NVFP4 stack
+
+
+def run_stack(args, world, rank, local):
+    """One step = the 30-layer NVFP4 stack over T=2048 tokens."""
+    import torch
+
+    from mixture_experts_transformer_b200 import binding as B
+    from mixture_experts_transformer_b200 import block, build
+    from mixture_experts_transformer_b200 import stack as stk
+
+    if rank == 0:
+        build.build()
+    barrier(world)
+    B.lib()
+    torch.cuda.set_device(local)
+    wl = WORKLOADS["nvfp4_stack"]
+    T, L = wl["T"], (args.layers or wl["layers"])
+    gcal = torch.Generator(device="cuda").manual_seed(2)
+    x_calib = torch.empty((256, D), device="cuda").normal_(0.0, 1.0, generator=gcal).to(torch.bfloat16)
+    st, kept = stk.build_stack(
+        lambda l: gen_weights_gpu(seed=l), L, x_calib, keep_bf16=set(range(min(L, 2))) if world == 1 else None
+    )
+    gx = torch.Generator(device="cuda").manual_seed(1 + rank)
+    x = torch.empty((T, D), device="cuda").normal_(0.0, 1.0, generator=gx).to(torch.bfloat16)
+    ws = stk.stack_workspace(st, T)
+    bufs = [torch.empty((T, D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    stream = torch.cuda.current_stream()
+
+    # touched experts per layer (routing statistics, outside the timed region)
+    touched = []
+    cur = x
+    for l in range(L):
+        r = block.forward_nvfp4(st.layers[l], cur, st.scales[l], rms_norm_out=True, debug=True, workspace=ws)
+        touched.append(int((r.cnt > 0).sum().item()))
+        cur = r.out.clone()
+    if B.moe_get_device_status() != B.MOE_OK:
+        raise RuntimeError("device status after the debug pass")
+
+    for _ in range(args.warmup):
+        stk.stack_forward(st, x, bufs, ws, stream)
+    torch.cuda.synchronize()
+    launches_per_step = 0
+    B.moe_profile_begin()
+    stk.stack_forward(st, x, bufs, ws, stream)
+    torch.cuda.synchronize()
+    breakdown = B.moe_profile_end()
+    launches_per_step = sum(v[1] for v in breakdown.values())
+    dominant = max(breakdown, key=lambda k: breakdown[k][0])
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        B.moe_profile_begin([dominant])
+        e0.record(stream)
+        for _ in range(args.steps):
+            stk.stack_forward(st, x, bufs, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_kernel = B.moe_profile_end()
+    barrier(world)
+    ms = reduce_max(e0.elapsed_time(e1), world)
+    agg = aggregate(T, args.steps, ms, world)
+    if B.moe_get_device_status() != B.MOE_OK:
+        raise RuntimeError("device status after the timed region")
+
+    # end to end: host tokens in, host tokens out, through the library per layer
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        r = stk.stack_forward(st, x_dev, bufs, ws, stream)
+        out_host.copy_(r.out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(t0.elapsed_time(t1), world)
+    barrier(world)
+    if rank != 0:
+        return None
+
+    peaks = measured_peaks()
+    step_ms = agg["ms_per_step"]
+    dom_ms = per_kernel[dominant][0] / per_kernel[dominant][1]
+    mean_touched = float(np.mean(touched))
+    dims = st.dims
+    lin = lambda K, N: N * K // 2 + ((N + 127) // 128) * (K // 64) * 512  # noqa: E731
+    R = T * K_TOP
+    if dominant == "fp4_gemm_gateup":
+        byts = mean_touched * 2 * lin(D, F) + 2 * lin(D, S) + (R + T) * (D // 2 + D // 16) + (R * F + T * S) * 9 // 16
+    elif dominant == "fp4_gemm_down":
+        byts = mean_touched * lin(F, D) + lin(S, D) + (R * F + T * S) * 9 // 16 + R * D * 2 + T * D * 4
+    else:
+        byts, _ = algorithmic(dominant, T, int(mean_touched), None)
+    weight_bytes = sum(stk.fp4_weight_bytes(dims, t) for t in touched) + L * ROUTER_BYTES
+    fp4_peak = peaks["bf16_tflops"] * FP4_TFLOPS_NOMINAL_RATIO
+    gemm_flops = L * T * FLOP_PER_TOKEN_GEMM
+    res = {
+        "metric": METRIC,
+        "value": agg["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e2m1, e4m3 group scales, fp32 accumulate; router bf16)",
+        "data": "synthetic: seeded N(0,0.02) random-init weights per layer (seed = layer), x ~ N(0,1)",
+        "config": {
+            "workload": wl["desc"] if L == 30 else wl["desc"].replace("30 ", f"{L} "),
+            "tokens_per_gpu": T,
+            "layers": L,
+            "global_batch": T * world,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (13 GB of NVFP4 weights per step)",
+            "calibration": "static activation scales from a 256-token batch (seed 2) through the stack",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": dominant,
+            "achieved": byts / (dom_ms / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"],
+            "peak_source": f"{peaks['source']} hbm_gbs",
+            "unit": "GB/s",
+            "frac": byts / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "traffic": ncu_traffic(dominant, "nvfp4_stack"),
+            "algorithmic_bytes": byts,
+            "kernel_ms": dom_ms,
+        },
+        "block_roofline": {
+            "hbm_weights_gbs": weight_bytes / (step_ms / 1e3) / 1e9,
+            "hbm_frac": weight_bytes / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "fp4_tensor_tflops": gemm_flops / (step_ms / 1e3) / 1e12,
+            "fp4_tensor_frac": gemm_flops / (step_ms / 1e3) / 1e12 / fp4_peak,
+            "fp4_peak_tflops": fp4_peak,
+            "fp4_peak_source": "measured bf16 burst x nominal fp4:bf16 ratio 4",
+            "touched_experts_mean": mean_touched,
+        },
+        "kernels_ms_per_launch": {k: v[0] / v[1] for k, v in breakdown.items()},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {
+            "value": T * args.steps * world / (e2e_ms / 1e3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": T * D * 2,
+            "d2h_bytes_per_step": T * D * 2,
+        },
+        "clocks": clocks.report(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_stack(kept, x, L)
+    return res
+
+
+def cpu_baseline_stack(kept, x, n_layers, budget_s=12.0):
+    """The oracle's NVFP4 block on one token through the first kept layers,
+    scaled to the whole stack (per-token, per-layer time x layers)."""
+    from oracle import moe_oracle as mo
+    from oracle import nvfp4 as nv
+
+    xb = x[:1].cpu().view(__import__("torch").int16).numpy().view(np.uint16)
+    hosts = [_host_weights(kept[l]) for l in sorted(kept)]
+    scales = [nv.act_scales_from_calibration(xb, *(h.w_router, h.wg, h.wu, h.wd, h.sg, h.su, h.sd)) for h in hosts]
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        cur = xb
+        for h, sc in zip(hosts, scales):
+            out = nv.moe_block_nvfp4(cur, h.w_router, h.wg, h.wu, h.wd, h.sg, h.su, h.sd, *sc)["out"]
+            from mixture_experts_transformer_b200 import inputs
+
+            cur = inputs.f32_to_bf16_bits(mo.rms_normalize(out).astype(np.float32))
+            n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    per_token_layer = el / n
+    return {
+        "value": 1.0 / (per_token_layer * n_layers),
+        "unit": "tokens/s",
+        "cores": _oracle_cores(),
+        "kind": "oracle",
+        "sample": f"1 token through layers {sorted(kept)} of the stack {n} times in {el:.1f} s, scaled to {n_layers} layers",
+    }
+
+
 # ----------------------------------------------------------- CPU oracle
 
 
@@ -527,6 +734,8 @@ def main():
     try:
         if args.impl == "reference":
             res = run_reference(args, world, rank)
+        elif args.workload == "nvfp4_stack":
+            res = run_stack(args, world, rank, local)
         else:
             res = run_ours(args, world, rank, local)
         if rank == 0 and res is not None:

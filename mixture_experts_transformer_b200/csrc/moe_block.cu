@@ -376,7 +376,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S, d.D, base, cnt, off,
                                                   reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                                   reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                                  reinterpret_cast<TileCounts*>(ws + L.counts), 0);
+                                                  reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
@@ -600,7 +600,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256);
     MOE_TRY(ls_.done(le_));
   }
   {
@@ -632,7 +632,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   {
     LaunchScope ls_(kKFp4GateUp, st);
     const cudaError_t le_ =
-        launch_k(fp4_gemm_kernel<true>, std::min(s->sm_count, L.max_tiles_gu), kGemmThreads, kF4SmemBytes, st, gu);
+        launch_k(fp4_gemm_kernel<true>, std::min(s->sm_count, L.max_tiles_gu), kF4Threads, kF4SmemBytes, st, gu);
     MOE_TRY(ls_.done(le_));
   }
 
@@ -655,7 +655,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   {
     LaunchScope ls_(kKFp4Down, st);
     const cudaError_t le_ =
-        launch_k(fp4_gemm_kernel<false>, std::min(s->sm_count, L.max_tiles_dn), kGemmThreads, kF4SmemBytes, st, dn);
+        launch_k(fp4_gemm_kernel<false>, std::min(s->sm_count, L.max_tiles_dn), kF4Threads, kF4SmemBytes, st, dn);
     MOE_TRY(ls_.done(le_));
   }
   {

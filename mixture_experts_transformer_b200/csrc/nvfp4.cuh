@@ -20,11 +20,13 @@
 //
 // The GEMM (fp4_gemm_kernel) is the bf16 grouped GEMM's structure with
 // `tcgen05.mma.kind::mxf4nvf4.block_scale.block16`: TMA brings 256-K stages of
-// A and B codes plus the matching scale atoms (a bulk copy), the MMA thread
-// moves each 64-K step's scale atoms into TMEM with tcgen05.cp (32x128b,
-// broadcast to the four lane quarters) and issues two M=128, N=128 MMAs.
-// The epilogue multiplies by 1/(G_act * G_weight); the gate|up epilogue then
-// quantises the GeGLU rows h to NVFP4 for the down projection.
+// A and B codes plus the matching scale atoms (a bulk copy); per stage the MMA
+// thread first moves all of the stage's scale atoms into TMEM with tcgen05.cp
+// (32x128b, broadcast to the four lane quarters; the copies pipeline), then
+// issues two M=128, N=128 MMAs per 64-K step. Eight epilogue warps (two per
+// TMEM lane quarter, each half of the columns) multiply by 1/(G_act *
+// G_weight); the gate|up epilogue then quantises the GeGLU rows h to NVFP4 for
+// the down projection.
 #pragma once
 
 #include "grouped_gemm.cuh"
@@ -219,6 +221,7 @@ constexpr int kF4BBytes = 2 * 128 * 128;         // two 128-row blocks
 constexpr int kF4SfBytes = 4 * 512;              // 4 atoms (4 x 64 K) of one 128-row block
 constexpr int kF4Stages = 4;
 constexpr int kF4SfSlots = 16;                   // TMEM scale slots (ring over 64-K steps)
+constexpr int kF4Threads = 320;                  // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
 constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 1024 + 256;
 
 struct Fp4Problem {
@@ -291,6 +294,8 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Output columns of a tile: GATEUP 128 per projection (gate and up side by
+// side in the 256-column accumulator), DOWN 256.
 template <bool GATEUP>
 __device__ __forceinline__ int f4_tile_cols(const Fp4Problem& pr, int n0) {
   const int cap = GATEUP ? 128 : 256;
@@ -298,11 +303,13 @@ __device__ __forceinline__ int f4_tile_cols(const Fp4Problem& pr, int n0) {
   return rem < cap ? rem : cap;
 }
 
-// TMEM columns: accumulator [0, 256) (GATEUP: gate 0..127, up 128..255; DOWN:
-// output columns n0 .. n0+255), scale slots from 256: slot i holds the A
-// scales at +0, B block 0 at +4, B block 1 at +8.
+// TMEM columns [0, 256): one accumulator (GATEUP: gate 0..127, up 128..255;
+// DOWN: output columns n0 .. n0+255) - a second one would not leave room for
+// the scale slots, so the epilogue stages it in registers and releases it at
+// once. From 256: scale slots, slot i holding the A scales at +0, B block 0 at
+// +4, B block 1 at +8.
 template <bool GATEUP>
-__global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_constant__ Fp4Params P) {
+__global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_constant__ Fp4Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -311,9 +318,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
   uint8_t* sSfB = sSfA + kF4Stages * kF4SfBytes;  // per stage: block 0 atoms, then block 1 atoms
   uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + kF4Stages * 2 * kF4SfBytes);
   uint64_t* empty = full + kF4Stages;
+  constexpr int kAccStages = 1;
+  constexpr uint32_t kAccStride = 256;
   uint64_t* acc_full = empty + kF4Stages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -324,8 +333,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);  // one arrival per epilogue warp
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -424,7 +435,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
-      int s = 0, slot = 0;
+      int s = 0, slot = 0, acc = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool any = false;
       const uint32_t idesc = idesc_nvf4_m128(128);
@@ -436,8 +447,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
         const int k64 = pr.K / 64;
         const int nstage = (pr.K + kF4KStage - 1) / kF4KStage;
         const bool two_b = GATEUP || (tile.n0 + 128 < pr.N);
-        if (!mbar_wait(acc_empty, acc_ph ^ 1, abort_flag, P.err)) break;
+        if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag, P.err)) break;
         tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + acc * kAccStride;
         bool ok = true;
         for (int ks = 0; ks < nstage; ++ks) {
           if (!mbar_wait(&full[s], ph, abort_flag, P.err)) {
@@ -450,22 +462,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
           const uint32_t b_addr = smem_u32(sB + s * kF4BBytes);
           const uint32_t sfa_addr = smem_u32(sSfA + s * kF4SfBytes);
           const uint32_t sfb_addr = smem_u32(sSfB + (2 * s) * kF4SfBytes);
+          // the whole stage's scale atoms first (the copies pipeline), then its MMAs
           for (int i = 0; i < nks; ++i) {
-            const uint32_t cols = tmem_base + kAccCols + slot * 16;
+            const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
             tmem_cp_32x128b_x4(cols, sdesc_sf_atom(sfa_addr + i * 512));
             tmem_cp_32x128b_x4(cols + 4, sdesc_sf_atom(sfb_addr + i * 512));
             if (two_b) tmem_cp_32x128b_x4(cols + 8, sdesc_sf_atom(sfb_addr + kF4SfBytes + i * 512));
+          }
+          for (int i = 0; i < nks; ++i) {
+            const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
             // 64 K of e2m1 = 32 B per row inside the 128-byte swizzled rows
             const uint64_t ad = sdesc_sw128(a_addr + i * 32, 16, 1024);
             const uint64_t bd0 = sdesc_sw128(b_addr + i * 32, 16, 1024);
-            const uint32_t acc = (ks | i) != 0;
-            umma_nvf4(tmem_base, ad, bd0, idesc, cols, cols + 4, acc);
+            const uint32_t accum = (ks | i) != 0;
+            umma_nvf4(d_tmem, ad, bd0, idesc, cols, cols + 4, accum);
             if (two_b) {
               const uint64_t bd1 = sdesc_sw128(b_addr + kF4BBytes / 2 + i * 32, 16, 1024);
-              umma_nvf4(tmem_base + 128, ad, bd1, idesc, cols, cols + 8, acc);
+              umma_nvf4(d_tmem + 128, ad, bd1, idesc, cols, cols + 8, accum);
             }
-            slot = (slot + 1) % kF4SfSlots;
           }
+          slot = (slot + nks) % kF4SfSlots;
           any = true;
           umma_commit(&empty[s]);
           if (++s == kF4Stages) {
@@ -474,8 +490,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
           }
         }
         if (!ok) break;
-        umma_commit(acc_full);
-        acc_ph ^= 1;
+        umma_commit(&acc_full[acc]);
+        if (++acc == kAccStages) {
+          acc = 0;
+          acc_ph ^= 1;
+        }
       }
       if (any) {
         umma_commit(drain);
@@ -485,8 +504,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
     }
   } else {
     // ----------------------------------------------------------- epilogue
+    // warps 2..9: TMEM lane quarter warp % 4, column half (warp - 2) / 4
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
+    int acc_i = 0;
     uint32_t acc_ph = 0;
     for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
       const Tile tile = P.tiles[ti];
@@ -494,22 +516,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
       if (p >= P.nprob) break;
       const Fp4Problem& pr = P.prob[p];
       const int wn = f4_tile_cols<GATEUP>(pr, tile.n0);
-      const bool ready = mbar_wait(acc_full, acc_ph, abort_flag, P.err);
+      const bool ready = mbar_wait(&acc_full[acc_i], acc_ph, abort_flag, P.err);
       __syncwarp();
       if (!ready) break;
       tc_fence_after_sync();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t tbase = tmem_base + acc_i * kAccStride + (static_cast<uint32_t>(quarter * 32) << 16);
       const bool valid = r < tile.rows;
       const int grow = tile.row0 + r;
+      // Bring this thread's accumulator columns into registers and hand TMEM
+      // back at once, so the next tile's MMAs overlap the math and stores below.
+      // Column chunks of 32: j = half * 32 + 64 c (c = 0..3 while j < wn).
+      uint32_t acc[4][32];
+#pragma unroll
+      for (int c = 0; c < (GATEUP ? 2 : 4); ++c) {
+        const int j = half * 32 + 64 * c;
+        if (j < wn) {
+          tmem_ld_32x32b_x32(tbase + j, acc[c]);
+          if (GATEUP) tmem_ld_32x32b_x32(tbase + 128 + j, acc[2 + c]);
+        }
+      }
+      tmem_ld_wait();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc_i]);
+      if (++acc_i == kAccStages) {
+        acc_i = 0;
+        acc_ph ^= 1;
+      }
       if (GATEUP) {
         const float ag = 1.0f / (pr.ga * pr.gb0[g]);
         const float au = 1.0f / (pr.ga * pr.gb1[g]);
         uint8_t* q = reinterpret_cast<uint8_t*>(pr.out) + static_cast<size_t>(grow) * (pr.N / 2);
-        for (int j = 0; j < wn; j += 32) {
-          uint32_t gv[32], uv[32];
-          tmem_ld_32x32b_x32(tbase + j, gv);
-          tmem_ld_32x32b_x32(tbase + 128 + j, uv);
-          tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int j = half * 32 + 64 * c;
+          if (j >= wn) continue;
           uint2 codes[2];
           uint32_t sc[2];
 #pragma unroll
@@ -517,7 +558,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
             float v[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              v[i] = gelu_tanh(__uint_as_float(gv[16 * h + i]) * ag) * (__uint_as_float(uv[16 * h + i]) * au);
+              v[i] = gelu_tanh(__uint_as_float(acc[c][16 * h + i]) * ag) *
+                     (__uint_as_float(acc[2 + c][16 * h + i]) * au);
             sc[h] = nvfp4_group(v, pr.g_out, &codes[h]);
           }
           if (valid) {
@@ -527,38 +569,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) fp4_gemm_kernel(const __grid_
             pr.out_sf[sf_offset(grow, c16 + 1, pr.N / 64)] = static_cast<uint8_t>(sc[1]);
           }
         }
-      } else {
+      } else if (valid) {
         const float alpha = 1.0f / (pr.ga * pr.gb0[g]);
-        for (int j = 0; j < wn; j += 32) {
-          uint32_t a[32];
-          tmem_ld_32x32b_x32(tbase + j, a);
-          tmem_ld_wait();
-          if (valid) {
-            if (pr.out_f32) {
-              float4* dst =
-                  reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(__uint_as_float(a[4 * v]) * alpha, __uint_as_float(a[4 * v + 1]) * alpha,
-                                     __uint_as_float(a[4 * v + 2]) * alpha, __uint_as_float(a[4 * v + 3]) * alpha);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) +
-                                                    static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
+        for (int c = 0; c < 4; ++c) {
+          const int j = half * 32 + 64 * c;
+          if (j >= wn) continue;
+          const uint32_t* a = acc[c];
+          if (pr.out_f32) {
+            float4* dst =
+                reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
 #pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(
-                    pack_bf16x2(__uint_as_float(a[8 * v]) * alpha, __uint_as_float(a[8 * v + 1]) * alpha),
-                    pack_bf16x2(__uint_as_float(a[8 * v + 2]) * alpha, __uint_as_float(a[8 * v + 3]) * alpha),
-                    pack_bf16x2(__uint_as_float(a[8 * v + 4]) * alpha, __uint_as_float(a[8 * v + 5]) * alpha),
-                    pack_bf16x2(__uint_as_float(a[8 * v + 6]) * alpha, __uint_as_float(a[8 * v + 7]) * alpha));
-            }
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(a[4 * v]) * alpha, __uint_as_float(a[4 * v + 1]) * alpha,
+                                   __uint_as_float(a[4 * v + 2]) * alpha, __uint_as_float(a[4 * v + 3]) * alpha);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) +
+                                                  static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(
+                  pack_bf16x2(__uint_as_float(a[8 * v]) * alpha, __uint_as_float(a[8 * v + 1]) * alpha),
+                  pack_bf16x2(__uint_as_float(a[8 * v + 2]) * alpha, __uint_as_float(a[8 * v + 3]) * alpha),
+                  pack_bf16x2(__uint_as_float(a[8 * v + 4]) * alpha, __uint_as_float(a[8 * v + 5]) * alpha),
+                  pack_bf16x2(__uint_as_float(a[8 * v + 6]) * alpha, __uint_as_float(a[8 * v + 7]) * alpha));
           }
         }
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
-      acc_ph ^= 1;
+
     }
   }
 

@@ -45,7 +45,8 @@ __global__ void build_masks_kernel(const int32_t* __restrict__ idx, int T, int k
 }
 
 // One CTA of 1024 threads: thread (e, seg) walks one eighth of the 32-token
-// chunks of expert e. Produces cnt, off, base[c][e] and the tile lists:
+// chunks of expert e. Produces cnt, off, base[c][e] and the tile lists
+// (gate|up tiles 128 output columns per projection, down tiles dn_cols wide):
 // shared-MLP tiles first (problem 1), then expert tiles (problem 0) expert by
 // expert, column tile, then row tile, so CTAs that run at the same time read
 // the same weight columns and share them through L2.
@@ -56,7 +57,8 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
                                                                   int32_t* __restrict__ off_out,
                                                                   Tile* __restrict__ tiles_gu,
                                                                   Tile* __restrict__ tiles_dn,
-                                                                  TileCounts* __restrict__ counts, int padded) {
+                                                                  TileCounts* __restrict__ counts, int padded,
+                                                                  int dn_cols) {
   __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   const int mt_sh = (T + kBM - 1) / kBM;
   const int nt_gu_sh = (S + 127) / 128;
   const int nt_gu = (F + 127) / 128;
-  const int nt_dn = (D + 255) / 256;
+  const int nt_dn = (D + dn_cols - 1) / dn_cols;
   const int n_sh_gu = nt_gu_sh * mt_sh;
   const int n_sh_dn = nt_dn * mt_sh;
   for (int i = threadIdx.x; i < n_sh_gu; i += kScanThreads) {
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   }
   for (int i = threadIdx.x; i < n_sh_dn; i += kScanThreads) {
     const int nt = i / mt_sh, m = i % mt_sh;
-    tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * 256};
+    tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * dn_cols};
   }
   if (e < E && c_e > 0) {
     const int mt = (c_e + kBM - 1) / kBM;
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     }
     for (int i = seg; i < nt_dn * mt; i += kScanSegs) {
       const int nt = i / mt, m = i % mt;
-      tiles_dn[base_dn + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * 256};
+      tiles_dn[base_dn + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * dn_cols};
     }
   }
   if (threadIdx.x == 0) {
