@@ -119,8 +119,8 @@ typedef struct moe_params {
 
 /*
  * Where the block's intermediates live inside a workspace (byte offsets from
- * its start; a size of 0 means the buffer is unused). R = T * top_k routed
- * rows, ordered expert by expert, tokens ascending within an expert.
+ * its start). R = T * top_k routed rows, ordered expert by expert, tokens
+ * ascending within an expert.
  *   x_perm [R, embed_dim] bf16   - x gathered into routed-row order
  *   h      [R, expert_dim] bf16  - routed GeGLU hidden rows
  *   y      [R, embed_dim] bf16   - routed expert outputs (unweighted)

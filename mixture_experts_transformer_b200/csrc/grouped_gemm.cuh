@@ -9,11 +9,12 @@
 // N contiguous (the weights exactly as given), which the tensor core reads as
 // an MN-major operand, so no weight is repacked.
 //
-// Roles (192 threads, one CTA per SM):
+// Roles (320 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile 128x64 and B chunks 64(K)x64(N) per stage
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
-//   warps 2..5  epilogue: tcgen05.ld the fp32 accumulator, apply GeGLU or
-//               convert, store rows that belong to the tile
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (each half of the
+//               column chunks): tcgen05.ld the fp32 accumulator, apply GeGLU
+//               or convert, store rows that belong to the tile
 // Shared memory: 4 stages x (16 KB A + 32 KB B), 128-byte swizzle.
 // TMEM: 2 accumulator buffers x 256 fp32 columns, so the epilogue of one tile
 // overlaps the main loop of the next.
@@ -22,6 +23,14 @@
 // of the up weights side by side in shared memory, so ONE MMA of N = 2*wn
 // computes both projections of wn output columns (wn = 128, or 64 for the
 // last columns): TMEM columns [0, wn) hold x Bg, [wn, 2 wn) hold x Bu.
+//
+// PAIRED (large batches): a tile carries two 128-row blocks of the same
+// expert and column tile; each stage holds both A blocks and one B, the MMA
+// thread issues two M=128 MMAs per K step into two 256-column accumulators,
+// and epilogue warps 2..5 / 6..9 drain one each. Sharing B cuts the bytes per
+// FLOP by a third and 3 stages of 64 KB keep ~1.6 us of loads in flight, which
+// is what lets the tensor cores run at their rate instead of waiting on data.
+// The accumulators then fill TMEM, so they are single-buffered.
 #pragma once
 
 #include "ptx.cuh"
@@ -37,22 +46,25 @@ constexpr int kMaxBChunks = 4;
 constexpr int kBStageBytes = kMaxBChunks * kBChunkBytes;
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
 constexpr int kGemmSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 /*align*/ + 256 /*barriers*/;
 
 // One 128-row work tile. pg = (problem << 16) | group.
 struct Tile {
   int32_t pg;
-  int32_t row0;  // first A row
-  int32_t rows;  // rows of A that belong to this tile (1..128)
-  int32_t n0;    // first output column (per projection for GATEUP)
+  int32_t row0;   // first A row
+  int32_t rows;   // rows of A that belong to this tile (1..128)
+  int32_t n0;     // first output column (per projection for GATEUP)
+  int32_t row1;   // PAIRED: first row of the second 128-row block
+  int32_t rows1;  // PAIRED: its rows (0: no second block)
+  int32_t pad[2];
 };
 
 struct GemmProblem {
   int K;        // reduction length, multiple of 64
   int N;        // output columns, multiple of 64
   int groups;   // number of B matrices (range check)
-  int a_rows;   // rows of A (range check)
+  int a_rows;   // rows of the tiles' row space (range check)
   void* out;    // [a_rows, ldo] bf16 or fp32
   int ldo;
   int out_f32;
@@ -76,12 +88,15 @@ __device__ __forceinline__ int tile_cols(const GemmProblem& pr, int n0) {
   return rem < cap ? rem : cap;
 }
 
-template <bool GATEUP>
+template <bool GATEUP, bool PAIRED = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams P) {
+  constexpr int kSt = PAIRED ? 3 : kStages;
+  constexpr int kAS = PAIRED ? 2 * kAStageBytes : kAStageBytes;
+  static_assert(kSt * (kAS + kBStageBytes) <= kStages * (kAStageBytes + kBStageBytes), "shared memory budget");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kStages * kAStageBytes;
+  uint8_t* sB = smem + kSt * kAS;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * (kAStageBytes + kBStageBytes));
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -100,7 +115,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[a], PAIRED ? 4 : 8);  // one arrival per epilogue warp draining it
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -127,65 +142,72 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   const int num_tiles = *P.num_tiles;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------ TMA producer
-      int s = 0;
-      uint32_t ph = 0;
-      int issued = 0;
-      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
-        const Tile tile = P.tiles[ti];
-        const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
-        if (p >= P.nprob) {
+    // -------------------------------------------------------- TMA producer
+    // The whole warp walks the tiles; lane 0 arms each stage's barrier and
+    // issues the loads.
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      const Tile tile = P.tiles[ti];
+      const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+      const bool bad_p = p >= P.nprob;
+      const GemmProblem& pr = P.prob[bad_p ? 0 : p];
+      const bool has1 = PAIRED && tile.rows1 > 0;
+      if (bad_p || g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || tile.rows < 1 || tile.rows > kBM ||
+          tile.n0 < 0 || tile.n0 >= pr.N || (has1 && (tile.row1 < 0 || tile.row1 >= pr.a_rows || tile.rows1 > kBM))) {
+        if (lane == 0) {
           atomicOr(P.err, kErrBadTile);
           *abort_flag = 1;
+        }
+        break;
+      }
+      const int wn = tile_cols<GATEUP>(pr, tile.n0);
+      const int cpp = wn >> 6;  // 64-column chunks per projection
+      const int nch = GATEUP ? 2 * cpp : cpp;
+      const uint32_t bytes = (has1 ? 2 : 1) * kAStageBytes + nch * kBChunkBytes;
+      const int nkb = pr.K / kBK;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        int waited = 1;
+        if (lane == 0) {
+          waited = mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err);
+          if (waited) mbar_arrive_expect_tx(&full[s], bytes);
+        }
+        if (!__shfl_sync(0xffffffffu, waited, 0)) {
+          ok = false;
           break;
         }
-        const GemmProblem& pr = P.prob[p];
-        if (g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || tile.n0 < 0 || tile.n0 >= pr.N) {
-          atomicOr(P.err, kErrBadTile);
-          *abort_flag = 1;
-          break;
-        }
-        const int wn = tile_cols<GATEUP>(pr, tile.n0);
-        const int cpp = wn >> 6;  // 64-column chunks per projection
-        const int nch = GATEUP ? 2 * cpp : cpp;
-        const uint32_t bytes = kAStageBytes + nch * kBChunkBytes;
-        const int nkb = pr.K / kBK;
-        bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d(sA + s * kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row0);
+        if (lane == 0) {
+          tma_load_2d(sA + s * kAS, &P.tmA[p], &full[s], kb * kBK, tile.row0);
+          if (has1) tma_load_2d(sA + s * kAS + kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row1);
           for (int c = 0; c < nch; ++c) {
             const bool up = GATEUP && c >= cpp;
             const int col = tile.n0 + (up ? c - cpp : c) * 64;
             tma_load_3d(sB + s * kBStageBytes + c * kBChunkBytes, up ? &P.tmB1[p] : &P.tmB0[p], &full[s], col,
                         kb * kBK, g);
           }
-          ++issued;
-          if (++s == kStages) {
-            s = 0;
-            ph ^= 1;
-          }
         }
-        if (!ok) break;
+        ++issued;
+        if (++s == kSt) {
+          s = 0;
+          ph ^= 1;
+        }
       }
-      if (*abort_flag) {
-        // let copies already in flight land before the CTA's memory goes away
-        int st = s;
-        uint32_t sp = ph;
-        const int pending = issued < kStages ? issued : kStages;
-        for (int i = 0; i < pending; ++i) {
-          if (--st < 0) {
-            st = kStages - 1;
-            sp ^= 1;
-          }
-          uint32_t dummy = 0;
-          mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
+      if (!ok) break;
+    }
+    __syncwarp();
+    if (lane == 0 && *abort_flag) {
+      // let copies already in flight land before the CTA's memory goes away
+      int st = s;
+      uint32_t sp = ph;
+      const int pending = issued < kSt ? issued : kSt;
+      for (int i = 0; i < pending; ++i) {
+        if (--st < 0) {
+          st = kSt - 1;
+          sp ^= 1;
         }
+        uint32_t dummy = 0;
+        mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -203,7 +225,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         const int n_mma = GATEUP ? 2 * wn : wn;
         const uint32_t idesc = idesc_bf16_m128(n_mma, 1);
         const int nkb = pr.K / kBK;
+        const bool has1 = PAIRED && tile.rows1 > 0;
         if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag, P.err)) break;
+        if (PAIRED && !mbar_wait(&acc_empty[1], acc_ph ^ 1, abort_flag, P.err)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         bool ok = true;
@@ -213,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(sA + s * kAStageBytes);
+          const uint32_t a_addr = smem_u32(sA + s * kAS);
           const uint32_t b_addr = smem_u32(sB + s * kBStageBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
@@ -223,17 +247,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             // chunks are 8 KB apart (LBO); +16 K-rows = +2048 B.
             const uint64_t bd = sdesc_sw128(b_addr + k * 2048, kBChunkBytes, 1024);
             umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            if (has1) umma_f16(tmem_base + kAccCols, sdesc_sw128(a_addr + kAStageBytes + k * 32, 16, 1024), bd, idesc,
+                               (kb | k) != 0);
           }
           any = true;
           umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
-          if (++s == kStages) {
+          if (++s == kSt) {
             s = 0;
             ph ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&acc_full[acc]);  // accumulator complete
-        if (++acc == 2) {
+        umma_commit(&acc_full[acc]);  // accumulator(s) complete
+        if (PAIRED) {
+          acc_ph ^= 1;
+        } else if (++acc == 2) {
           acc = 0;
           acc_ph ^= 1;
         }
@@ -248,7 +276,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   } else {
     // ----------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter..+31
+    const int half = (warp - 2) >> 2;  // unpaired: column chunks j = 32 * half + 64 c; PAIRED: the accumulator
     const int r = quarter * 32 + lane;
+    const int j_first = PAIRED ? 0 : 32 * half;
+    const int j_step = PAIRED ? 32 : 64;
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
@@ -261,12 +292,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       __syncwarp();
       if (!ready) break;
       tc_fence_after_sync();
-      const uint32_t tbase = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
-      const bool valid = r < tile.rows;
-      const size_t grow = static_cast<size_t>(tile.row0 + r);
+      const int a_id = PAIRED ? half : acc;  // accumulator this warp drains
+      const uint32_t tbase = tmem_base + a_id * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
+      const int t_rows = (PAIRED && half) ? tile.rows1 : tile.rows;
+      const int t_row0 = (PAIRED && half) ? tile.row1 : tile.row0;
+      const bool valid = r < t_rows;
+      const size_t grow = static_cast<size_t>(t_row0 + r);
+      if (!(PAIRED && half && t_rows <= 0)) {
       if (GATEUP) {
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo + tile.n0;
-        for (int j = 0; j < wn; j += 32) {
+        for (int j = j_first; j < wn; j += j_step) {
           uint32_t g[32], u[32];
           tmem_ld_32x32b_x32(tbase + j, g);
           tmem_ld_32x32b_x32(tbase + wn + j, u);
@@ -285,7 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           }
         }
       } else {
-        for (int j = 0; j < wn; j += 32) {
+        for (int j = j_first; j < wn; j += j_step) {
           uint32_t a[32];
           tmem_ld_32x32b_x32(tbase + j, a);
           tmem_ld_wait();
@@ -309,10 +344,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           }
         }
       }
+      }  // end of the drained accumulator's work
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      if (++acc == 2) {
+      if (lane == 0) mbar_arrive(&acc_empty[PAIRED ? half : acc]);
+      if (PAIRED) {
+        acc_ph ^= 1;
+      } else if (++acc == 2) {
         acc = 0;
         acc_ph ^= 1;
       }

@@ -42,6 +42,9 @@ struct Layout {
   int nsplit, nchunks, max_tiles_gu, max_tiles_dn;
 };
 
+// Large batches (experts average >= 160 routed rows) use the paired gate|up GEMM.
+bool paired_gateup(const Dims& d) { return static_cast<long long>(d.T) * d.k >= 160LL * d.E; }
+
 int router_splits(const Dims& d) {
   const int tiles = std::max(1, (d.T + kRouterTokens - 1) / kRouterTokens);
   int ns = (2 * kSmCountHint + tiles - 1) / tiles;
@@ -138,6 +141,9 @@ moe_status device_state(DeviceState** out) {
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kGemmSmemBytes) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(grouped_gemm_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaFuncSetAttribute(fp4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
@@ -366,25 +372,25 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
   return ls_.done(le_);
 }
 
-// Scan of the bitmasks, then the scatter (and, with x, the gather into x_perm).
+// Scan of the bitmasks, then the scatter (and, with x, the copy into x_perm).
 moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const int32_t* idx, const void* x,
                            int32_t* cnt, int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st) {
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(ws + L.masks);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   {
     LaunchScope ls_(kKRouteScan, st);
-    const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S, d.D, base, cnt, off,
-                                                  reinterpret_cast<Tile*>(ws + L.tiles_gu),
-                                                  reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                                  reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256);
+    const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
+                                     d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
+                                     reinterpret_cast<Tile*>(ws + L.tiles_dn),
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256, paired_gateup(d) ? 1 : 0);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
   const int blocks = static_cast<int>(std::min<long long>((R + 7) / 8, 148LL * 64));
   LaunchScope ls_(kKRouteScatter, st);
   const cudaError_t le_ = launch_k(route_scatter_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E, d.D,
-                                               static_cast<const __nv_bfloat16*>(x), row_of, token_of,
-                                               reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm));
+                                   static_cast<const __nv_bfloat16*>(x), row_of, token_of,
+                                   reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm));
   return ls_.done(le_);
 }
 
@@ -397,11 +403,11 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   int32_t* off = reinterpret_cast<int32_t*>(ws + L.off);
   int32_t* row_of = reinterpret_cast<int32_t*>(ws + L.row_of);
   int32_t* token_of = reinterpret_cast<int32_t*>(ws + L.token_of);
-  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
   __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
   __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
   __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(ws + L.hs);
   float* sbuf = reinterpret_cast<float*>(ws + L.s);
+  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
   const TileCounts* counts = reinterpret_cast<const TileCounts*>(ws + L.counts);
 
   MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
@@ -423,7 +429,9 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   const int grid_gu = std::min(s->sm_count, L.max_tiles_gu);
   {
   LaunchScope ls_(kKGemmGateUp, st);
-  const cudaError_t le_ = launch_k(grouped_gemm_kernel<true>, grid_gu, kGemmThreads, kGemmSmemBytes, st, gu);
+  const cudaError_t le_ =
+      paired_gateup(d) ? launch_k(grouped_gemm_kernel<true, true>, grid_gu, kGemmThreads, kGemmSmemBytes, st, gu)
+                       : launch_k(grouped_gemm_kernel<true>, grid_gu, kGemmThreads, kGemmSmemBytes, st, gu);
   MOE_TRY(ls_.done(le_));
   }
 
@@ -600,7 +608,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 0);
     MOE_TRY(ls_.done(le_));
   }
   {

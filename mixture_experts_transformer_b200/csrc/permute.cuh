@@ -58,10 +58,11 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
                                                                   Tile* __restrict__ tiles_gu,
                                                                   Tile* __restrict__ tiles_dn,
                                                                   TileCounts* __restrict__ counts, int padded,
-                                                                  int dn_cols) {
+                                                                  int dn_cols, int pair_gu) {
   __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
+  __shared__ int s_ptoff[129];  // prefix of gate|up row-tile pairs per expert
   __shared__ int s_cnt[128];
   pdl_wait_then_release();
   const int e = threadIdx.x & 127;
@@ -85,28 +86,34 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   __syncthreads();
   if (threadIdx.x < 32) {  // exclusive scans over experts, one warp
     const int lane = threadIdx.x;
-    int carry = 0, mcarry = 0;
+    int carry = 0, mcarry = 0, pcarry = 0;
     for (int b = 0; b < 128; b += 32) {
       const int v = s_cnt[b + lane];
       const int mv = (v + kBM - 1) / kBM;
-      int inc = v, minc = mv;
+      const int pv = pair_gu ? (mv + 1) / 2 : mv;
+      int inc = v, minc = mv, pinc = pv;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int a = __shfl_up_sync(0xffffffffu, inc, o);
         const int ma = __shfl_up_sync(0xffffffffu, minc, o);
+        const int pa = __shfl_up_sync(0xffffffffu, pinc, o);
         if (lane >= o) {
           inc += a;
           minc += ma;
+          pinc += pa;
         }
       }
       s_off[b + lane] = carry + inc - v;
       s_mtoff[b + lane] = mcarry + minc - mv;
+      s_ptoff[b + lane] = pcarry + pinc - pv;
       carry += __shfl_sync(0xffffffffu, inc, 31);
       mcarry += __shfl_sync(0xffffffffu, minc, 31);
+      pcarry += __shfl_sync(0xffffffffu, pinc, 31);
     }
     if (lane == 0) {
       s_off[E] = carry;
       s_mtoff[E] = mcarry;
+      s_ptoff[E] = pcarry;
     }
   }
   __syncthreads();
@@ -127,42 +134,50 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   }
   if (threadIdx.x == 0) off_out[E] = s_off[E];
 
+  // gate|up tiles take one 128-row block (pair_gu = 0) or two consecutive
+  // ones of the same expert and column tile (pair_gu = 1, the paired GEMM)
+  const int mstep = pair_gu ? 2 : 1;
   const int mt_sh = (T + kBM - 1) / kBM;
+  const int pt_sh = (mt_sh + mstep - 1) / mstep;
   const int nt_gu_sh = (S + 127) / 128;
   const int nt_gu = (F + 127) / 128;
   const int nt_dn = (D + dn_cols - 1) / dn_cols;
-  const int n_sh_gu = nt_gu_sh * mt_sh;
+  const int n_sh_gu = nt_gu_sh * pt_sh;
   const int n_sh_dn = nt_dn * mt_sh;
   for (int i = threadIdx.x; i < n_sh_gu; i += kScanThreads) {
-    const int nt = i / mt_sh, m = i % mt_sh;
-    tiles_gu[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * 128};
+    const int nt = i / pt_sh, m = (i % pt_sh) * mstep;
+    const int r1 = pair_gu ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
+    tiles_gu[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * 128, (m + 1) * kBM, r1, {0, 0}};
   }
   for (int i = threadIdx.x; i < n_sh_dn; i += kScanThreads) {
     const int nt = i / mt_sh, m = i % mt_sh;
-    tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * dn_cols};
+    tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
   }
   if (e < E && c_e > 0) {
     const int mt = (c_e + kBM - 1) / kBM;
-    const int base_gu = n_sh_gu + s_mtoff[e] * nt_gu;
+    const int pt = (mt + mstep - 1) / mstep;
+    const int base_gu = n_sh_gu + s_ptoff[e] * nt_gu;
     const int base_dn = n_sh_dn + s_mtoff[e] * nt_dn;
-    for (int i = seg; i < nt_gu * mt; i += kScanSegs) {
-      const int nt = i / mt, m = i % mt;
-      tiles_gu[base_gu + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * 128};
+    for (int i = seg; i < nt_gu * pt; i += kScanSegs) {
+      const int nt = i / pt, m = (i % pt) * mstep;
+      const int r1 = pair_gu ? max(0, min(kBM, c_e - (m + 1) * kBM)) : 0;
+      tiles_gu[base_gu + i] =
+          Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * 128, row_base + (m + 1) * kBM, r1, {0, 0}};
     }
     for (int i = seg; i < nt_dn * mt; i += kScanSegs) {
       const int nt = i / mt, m = i % mt;
-      tiles_dn[base_dn + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * dn_cols};
+      tiles_dn[base_dn + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
     }
   }
   if (threadIdx.x == 0) {
-    counts->gateup = n_sh_gu + s_mtoff[E] * nt_gu;
+    counts->gateup = n_sh_gu + s_ptoff[E] * nt_gu;
     counts->down = n_sh_dn + s_mtoff[E] * nt_dn;
   }
 }
 
 // One warp per (token, slot): its routed row from the bitmasks; lane 0 writes
 // row_of / token_of, and (when x is given) the warp copies x[t] into
-// x_perm[row] with 16-byte vectors.
+// x_perm[row] with 16-byte vectors, so the GEMM's A tiles are plain boxes.
 __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __restrict__ idx,
                                                             const uint32_t* __restrict__ masks,
                                                             const int32_t* __restrict__ base, int T, int k, int E,
