@@ -70,8 +70,10 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   const int c0 = static_cast<int>((static_cast<long long>(seg) * nchunks) / kScanSegs);
   const int c1 = static_cast<int>((static_cast<long long>(seg + 1) * nchunks) / kScanSegs);
   int part = 0;
-  if (e < E)
+  if (e < E) {
+#pragma unroll 8
     for (int c = c0; c < c1; ++c) part += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
+  }
   s_seg[seg][e] = part;
   __syncthreads();
   if (seg == 0) {
@@ -123,6 +125,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   const int row_base = padded ? s_mtoff[e] * kBM : s_off[e];
   if (e < E) {
     int run = row_base + s_seg[seg][e];
+#pragma unroll 8
     for (int c = c0; c < c1; ++c) {
       base[static_cast<size_t>(c) * E + e] = run;
       run += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
@@ -153,21 +156,38 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     const int nt = i / mt_sh, m = i % mt_sh;
     tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
   }
-  if (e < E && c_e > 0) {
-    const int mt = (c_e + kBM - 1) / kBM;
-    const int pt = (mt + mstep - 1) / mstep;
-    const int base_gu = n_sh_gu + s_ptoff[e] * nt_gu;
-    const int base_dn = n_sh_dn + s_mtoff[e] * nt_dn;
-    for (int i = seg; i < nt_gu * pt; i += kScanSegs) {
-      const int nt = i / pt, m = (i % pt) * mstep;
-      const int r1 = pair_gu ? max(0, min(kBM, c_e - (m + 1) * kBM)) : 0;
-      tiles_gu[base_gu + i] =
-          Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * 128, row_base + (m + 1) * kBM, r1, {0, 0}};
+  // expert tiles, spread over all threads (one expert may own most of them):
+  // flat index f -> expert by binary search over the tile-offset prefix
+  const int n_e_gu = s_ptoff[E] * nt_gu;
+  for (int f = threadIdx.x; f < n_e_gu; f += kScanThreads) {
+    int lo = 0, hi = E - 1;  // largest ex with s_ptoff[ex] * nt_gu <= f
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_ptoff[mid] * nt_gu <= f) lo = mid; else hi = mid - 1;
     }
-    for (int i = seg; i < nt_dn * mt; i += kScanSegs) {
-      const int nt = i / mt, m = i % mt;
-      tiles_dn[base_dn + i] = Tile{e, row_base + m * kBM, min(kBM, c_e - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
+    const int ex = lo;
+    const int ce = s_cnt[ex];
+    const int pt = s_ptoff[ex + 1] - s_ptoff[ex];
+    const int i = f - s_ptoff[ex] * nt_gu;
+    const int nt = i / pt, m = (i % pt) * mstep;
+    const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
+    const int r1 = pair_gu ? max(0, min(kBM, ce - (m + 1) * kBM)) : 0;
+    tiles_gu[n_sh_gu + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * 128, rb + (m + 1) * kBM, r1, {0, 0}};
+  }
+  const int n_e_dn = s_mtoff[E] * nt_dn;
+  for (int f = threadIdx.x; f < n_e_dn; f += kScanThreads) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_mtoff[mid] * nt_dn <= f) lo = mid; else hi = mid - 1;
     }
+    const int ex = lo;
+    const int ce = s_cnt[ex];
+    const int mt = s_mtoff[ex + 1] - s_mtoff[ex];
+    const int i = f - s_mtoff[ex] * nt_dn;
+    const int nt = i / mt, m = i % mt;
+    const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
+    tiles_dn[n_sh_dn + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
   }
   if (threadIdx.x == 0) {
     counts->gateup = n_sh_gu + s_ptoff[E] * nt_gu;
