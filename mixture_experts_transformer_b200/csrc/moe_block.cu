@@ -45,11 +45,13 @@ struct Layout {
 // Large batches (experts average >= 160 routed rows) use the paired gate|up GEMM.
 bool paired_gateup(const Dims& d) { return static_cast<long long>(d.T) * d.k >= 160LL * d.E; }
 
+// Splits of the router's reduction: enough (token tile, split) CTAs for one
+// wave at one CTA per SM, at least two 64-wide slices per split.
 int router_splits(const Dims& d) {
   const int tiles = std::max(1, (d.T + kRouterTokens - 1) / kRouterTokens);
-  int ns = (2 * kSmCountHint + tiles - 1) / tiles;
+  int ns = kSmCountHint / tiles;
   ns = std::min(ns, 22);
-  ns = std::min(ns, d.D / kRouterKChunk);
+  ns = std::min(ns, d.D / (2 * kRouterBK));
   return std::max(ns, 1);
 }
 
@@ -137,6 +139,9 @@ moe_status device_state(DeviceState** out) {
     s.sm_count = prop.multiProcessorCount;
     if (s.arch_ok) {
       if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), g_device_error) != cudaSuccess) return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kRouterSmemBytes) != cudaSuccess)
+        return MOE_ERR_CUDA;
       if (cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -358,12 +363,21 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
                          const float* bias, int32_t* idx, float* w, cudaStream_t st) {
   float* partial = reinterpret_cast<float*>(ws + L.partial);
   uint32_t* masks = reinterpret_cast<uint32_t*>(ws + L.masks);
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  RouterParams rp{};
+  if (!map_2d(&rp.tmX, x, d.T, d.D, kRouterTokens) || !map_3d(&rp.tmW, wr, 1, d.D, d.E)) return MOE_ERR_CUDA;
+  rp.partial = partial;
+  rp.masks = masks;
+  rp.err = s->err;
+  rp.T = d.T;
+  rp.D = d.D;
+  rp.E = d.E;
+  rp.nsplit = L.nsplit;
   const dim3 g1((d.T + kRouterTokens - 1) / kRouterTokens, L.nsplit);
   {
     LaunchScope ls_(kKRouterLogits, st);
-    const cudaError_t le_ = launch_k(router_logits_kernel, g1, kRouterThreads, 0, st, static_cast<const __nv_bfloat16*>(x),
-                                                        static_cast<const __nv_bfloat16*>(wr), partial, masks, d.T,
-                                                        d.D, d.E, L.nsplit);
+    const cudaError_t le_ = launch_k(router_logits_kernel, g1, kRouterThreads, kRouterSmemBytes, st, rp);
     MOE_TRY(ls_.done(le_));
   }
   LaunchScope ls_(kKRouterTopk, st);

@@ -1,5 +1,5 @@
-// Router: logits = x W_router in fp32 on the CUDA cores, then top-k
-// selection and the softmax of the kept logits.
+// Router: logits = x W_router on the tensor cores (bf16 products, fp32
+// accumulation), then top-k selection and the softmax of the kept logits.
 //
 // Follows the layer statement: softmax gating over the expert logits, the
 // top_k_experts largest kept, their weights renormalised to sum to one
@@ -18,140 +18,186 @@
 
 namespace moe {
 
-constexpr int kRouterTokens = 128;  // tokens per CTA tile
-constexpr int kRouterKChunk = 32;   // reduction elements staged per step
+constexpr int kRouterTokens = 128;  // tokens per CTA tile (the MMA's M)
+constexpr int kRouterBK = 64;       // reduction elements per pipeline stage
+constexpr int kRouterStages = 4;
 constexpr int kRouterThreads = 128;
+constexpr int kRouterAStage = kRouterTokens * kRouterBK * 2;  // 16 KB of x
+constexpr int kRouterBChunk = kRouterBK * 64 * 2;             // 8 KB: 64 K-rows x 64 experts
+constexpr int kRouterBStage = 2 * kRouterBChunk;              // up to 128 experts
+constexpr int kRouterSmemBytes = kRouterStages * (kRouterAStage + kRouterBStage) + 1024 + 256;
 constexpr int kMaskTokens = 32;     // tokens per bitmask word
 constexpr int kTopkWarps = 4;       // one warp per token
 
-__device__ __forceinline__ void ffma2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
-
-__device__ __forceinline__ unsigned long long dup2(float a) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
-  return r;
-}
-
-__device__ __forceinline__ float2 unpack2(unsigned long long v) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-  return r;
-}
+struct RouterParams {
+  CUtensorMap tmX;  // x [T, D] bf16, box 64 (K) x 128 (tokens), 128-byte swizzle
+  CUtensorMap tmW;  // W_router [1, D, E] bf16 (experts contiguous), box 64 x 64 x 1
+  float* partial;   // [nsplit][T][E] fp32
+  uint32_t* masks;  // [ceil(T / 32)][E], cleared here for top-k's atomicOr
+  uint32_t* err;
+  int T, D, E, nsplit;
+};
 
 // partial[split][t][e] = sum over this split's slice of d of x[t, d] W[d, e].
 //
-// CTA tile 128 tokens x 128 experts, 128 threads; a warp owns 32 tokens, and
-// lane (tg = lane / 8, eg = lane % 8) owns tokens tg*4 + {0..3, 16..19} of the
-// warp and experts eg*4 + 32n + {0..3} (n = 0..3): 8 x 16 fp32 accumulators
-// held as packed pairs, updated with fma.rn.f32x2 (two experts of one token
-// per instruction). Shared memory holds the chunk as fp32, x transposed
-// ([k][token]) and W as is ([k][expert]); per k a lane reads its 8 x values
-// (a broadcast within each group of 8 lanes) and its 16 W values (8 lanes read
-// 128 contiguous bytes), so the reads are conflict-free: 6 16-byte loads feed
-// 128 FMAs. Every accumulator sums its slice in increasing d, so the result is
-// deterministic. CTAs of split 0 also clear the token-expert bitmask words of
-// their tokens. Requires E % 8 == 0, E <= 128, D % 32 == 0.
-__global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const __nv_bfloat16* __restrict__ x,
-                                                                       const __nv_bfloat16* __restrict__ w,
-                                                                       float* __restrict__ partial,
-                                                                       uint32_t* __restrict__ masks, int T, int D,
-                                                                       int E, int nsplit) {
-  __shared__ __align__(16) float xs[kRouterKChunk][kRouterTokens];
-  __shared__ __align__(16) float ws[kRouterKChunk][128];
+// One CTA per (128-token tile, split of the reduction), 128 threads. Thread 0
+// streams the split's 64-wide slices of x (K-major) and W (read as an N-major
+// operand, so the weights are used exactly as stored) into a 4-stage ring by
+// TMA; thread 32 issues tcgen05.mma (M = 128 tokens, N = 64 or 128 experts,
+// K = 16 per instruction) into a 128-column fp32 TMEM accumulator; then the
+// four warps each read their 32 TMEM lanes (tokens) and write the partial
+// logits. The products of bf16 values are exact in fp32 and the accumulation
+// order inside a split is fixed by the hardware, so the result is
+// deterministic. Tokens past T and experts past E are zero-filled by the copy
+// engine and never stored. CTAs of split 0 also clear the token-expert bitmask
+// words of their tokens. Requires E % 8 == 0, E <= 128, D % 64 == 0.
+__global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const __grid_constant__ RouterParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kRouterStages * kRouterAStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRouterStages * (kRouterAStage + kRouterBStage));
+  uint64_t* empty = full + kRouterStages;
+  uint64_t* acc_full = empty + kRouterStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  pdl_wait_then_release();
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int tg = lane >> 3, eg = lane & 7;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * kRouterTokens;
   const int split = blockIdx.y;
-  if (split == 0) {
-    const int words = (min(T, t0 + kRouterTokens) - t0 + kMaskTokens - 1) / kMaskTokens;
-    for (int i = tid; i < words * E; i += kRouterThreads) masks[static_cast<size_t>(t0 / kMaskTokens) * E + i] = 0u;
+  const int nkb_all = P.D / kRouterBK;
+  const int kb0 = static_cast<int>((static_cast<long long>(split) * nkb_all) / P.nsplit);
+  const int kb1 = static_cast<int>((static_cast<long long>(split + 1) * nkb_all) / P.nsplit);
+  const int nch = (P.E + 63) >> 6;  // 64-expert chunks of B
+  const int n_mma = 64 * nch;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRouterStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&P.tmX);
+    tma_prefetch_desc(&P.tmW);
   }
-  const int nchunks = D / kRouterKChunk;
-  const int c_begin = static_cast<int>((static_cast<long long>(split) * nchunks) / nsplit);
-  const int c_end = static_cast<int>((static_cast<long long>(split + 1) * nchunks) / nsplit);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_then_release();
 
-  unsigned long long acc[8][8];  // [token][expert pair]
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int p = 0; p < 8; ++p) acc[i][p] = 0ull;
-
-  // global -> registers for the next chunk while the current one is consumed
-  uint4 xr[4], wr[4];
-  const int my_t = t0 + tid;  // staging: thread tid brings token t0 + tid
-  auto load_chunk = [&](int c) {
-    const int k0 = c * kRouterKChunk;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      xr[q] = make_uint4(0, 0, 0, 0);
-      if (my_t < T) xr[q] = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(my_t) * D + k0) + q);
-      const int v = tid + q * kRouterThreads;  // 32 rows x 16 vectors of 8 experts
-      const int r = v >> 4, c8 = v & 15;
-      wr[q] = make_uint4(0, 0, 0, 0);
-      if (c8 * 8 < E) wr[q] = __ldg(reinterpret_cast<const uint4*>(w + static_cast<size_t>(k0 + r) * E + c8 * 8));
-    }
-  };
-  auto store_chunk = [&]() {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&xr[q]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) xs[q * 8 + i][tid] = __bfloat162float(xb[i]);
-      const int v = tid + q * kRouterThreads;
-      const int r = v >> 4, c8 = v & 15;
-      const __nv_bfloat16* wb = reinterpret_cast<const __nv_bfloat16*>(&wr[q]);
-      *reinterpret_cast<float4*>(&ws[r][c8 * 8]) = make_float4(
-          __bfloat162float(wb[0]), __bfloat162float(wb[1]), __bfloat162float(wb[2]), __bfloat162float(wb[3]));
-      *reinterpret_cast<float4*>(&ws[r][c8 * 8 + 4]) = make_float4(
-          __bfloat162float(wb[4]), __bfloat162float(wb[5]), __bfloat162float(wb[6]), __bfloat162float(wb[7]));
-    }
-  };
-
-  const int a_col = warp * 32 + tg * 4;
-  if (c_begin < c_end) load_chunk(c_begin);
-  for (int c = c_begin; c < c_end; ++c) {
-    __syncthreads();  // the previous chunk's readers are done
-    store_chunk();
-    __syncthreads();
-    if (c + 1 < c_end) load_chunk(c + 1);
-#pragma unroll 4
-    for (int kk = 0; kk < kRouterKChunk; ++kk) {
-      const float4 a_lo = *reinterpret_cast<const float4*>(&xs[kk][a_col]);
-      const float4 a_hi = *reinterpret_cast<const float4*>(&xs[kk][a_col + 16]);
-      const float a[8] = {a_lo.x, a_lo.y, a_lo.z, a_lo.w, a_hi.x, a_hi.y, a_hi.z, a_hi.w};
-      unsigned long long b[8];
-#pragma unroll
-      for (int n = 0; n < 4; ++n) {
-        const ulonglong2 bb = *reinterpret_cast<const ulonglong2*>(&ws[kk][eg * 4 + 32 * n]);
-        b[2 * n] = bb.x;
-        b[2 * n + 1] = bb.y;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const unsigned long long ad = dup2(a[i]);
-#pragma unroll
-        for (int p = 0; p < 8; ++p) ffma2(acc[i][p], ad, b[p]);
-      }
-    }
+  if (split == 0 && warp >= 2) {  // warps 2 and 3, while the pipeline fills
+    const int words = (min(P.T, t0 + kRouterTokens) - t0 + kMaskTokens - 1) / kMaskTokens;
+    for (int i = threadIdx.x - 64; i < words * P.E; i += kRouterThreads - 64)
+      P.masks[static_cast<size_t>(t0 / kMaskTokens) * P.E + i] = 0u;
   }
 
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int t = t0 + a_col + (i & 3) + (i >> 2) * 16;
-    if (t >= T) continue;
-    float* dst = partial + (static_cast<size_t>(split) * T + t) * E;
-#pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      const int e = eg * 4 + 32 * n;
-      if (e >= E) continue;
-      const float2 lo = unpack2(acc[i][2 * n]), hi = unpack2(acc[i][2 * n + 1]);
-      *reinterpret_cast<float4*>(dst + e) = make_float4(lo.x, lo.y, hi.x, hi.y);
+  if (threadIdx.x == 0) {
+    // ------------------------------------------------------------ producer
+    const uint32_t bytes = kRouterAStage + nch * kRouterBChunk;
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err)) break;
+      mbar_arrive_expect_tx(&full[s], bytes);
+      tma_load_2d(sA + s * kRouterAStage, &P.tmX, &full[s], kb * kRouterBK, t0);
+      for (int c = 0; c < nch; ++c)
+        tma_load_3d(sB + s * kRouterBStage + c * kRouterBChunk, &P.tmW, &full[s], c * 64, kb * kRouterBK, 0);
+      ++issued;
+      if (++s == kRouterStages) {
+        s = 0;
+        ph ^= 1;
+      }
     }
+    if (*abort_flag) {
+      // let the copies in flight land before the CTA's shared memory goes away
+      const int pending = issued < kRouterStages ? issued : kRouterStages;
+      for (int i = 0; i < pending; ++i) {
+        if (--s < 0) {
+          s = kRouterStages - 1;
+          ph ^= 1;
+        }
+        uint32_t dummy = 0;
+        mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
+      }
+    }
+  } else if (threadIdx.x == 32) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_bf16_m128(n_mma, 1);
+    int s = 0;
+    uint32_t ph = 0;
+    bool any = false;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&full[s], ph, abort_flag, P.err)) break;
+      tc_fence_after_sync();
+      const uint32_t a_addr = smem_u32(sA + s * kRouterAStage);
+      const uint32_t b_addr = smem_u32(sB + s * kRouterBStage);
+#pragma unroll
+      for (int k = 0; k < kRouterBK / 16; ++k) {
+        // A: K-major rows of 128 B, 8-row groups 1024 B apart, +32 B per 16 K.
+        // B: N-major, 8 K-rows per 1024 B swizzle atom, 64-expert chunks 8 KB
+        // apart, +2048 B per 16 K.
+        umma_f16(tmem_base, sdesc_sw128(a_addr + k * 32, 16, 1024), sdesc_sw128(b_addr + k * 2048, kRouterBChunk, 1024),
+                 idesc, (kb != kb0 || k != 0) ? 1u : 0u);
+      }
+      any = true;
+      umma_commit(&empty[s]);
+      if (++s == kRouterStages) {
+        s = 0;
+        ph ^= 1;
+      }
+    }
+    if (any) {
+      umma_commit(acc_full);  // every MMA above has completed once this arrives
+    } else {
+      mbar_arrive(acc_full);  // empty split (never with D >= 64 * nsplit): the partials are zero
+    }
+    // even after an abort, no MMA may still be running when TMEM is released
+    uint32_t dummy = 0;
+    mbar_wait(acc_full, 0, reinterpret_cast<volatile int*>(&dummy), P.err);
+  }
+  __syncwarp();
+
+  // -------------------------------------------------------------- epilogue
+  const int arrived = mbar_wait(acc_full, 0, abort_flag, P.err) && !*abort_flag;
+  const bool ready = __all_sync(0xffffffffu, arrived);
+  if (ready && kb1 > kb0) {
+    tc_fence_after_sync();
+    const int t = t0 + warp * 32 + lane;
+    float* dst = P.partial + (static_cast<size_t>(split) * P.T + t) * P.E;
+    for (int j = 0; j < n_mma; j += 32) {
+      uint32_t a[32];
+      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + j, a);
+      tmem_ld_wait();
+      if (t < P.T) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          if (j + 4 * v < P.E)
+            *reinterpret_cast<float4*>(dst + j + 4 * v) =
+                make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]), __uint_as_float(a[4 * v + 2]),
+                            __uint_as_float(a[4 * v + 3]));
+        }
+      }
+    }
+  } else if (ready) {
+    const int t = t0 + warp * 32 + lane;
+    if (t < P.T)
+      for (int e = 0; e < P.E; e += 4)
+        *reinterpret_cast<float4*>(P.partial + (static_cast<size_t>(split) * P.T + t) * P.E + e) =
+            make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, 128);
   }
 }
 

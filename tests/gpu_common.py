@@ -29,7 +29,14 @@ OUT_TOL = 1e-2
 BF16_SLACK = 1.25
 ACC_SLACK = 2e-3
 GAP = 1e-4
-W_TOL = 2e-6
+# Routing weights. Requiring exact expert sets wherever the oracle's logit gap
+# exceeds GAP presumes the kernel's logits agree with the oracle's to well
+# under GAP; the tensor cores accumulate the router's products in fp32 in their
+# own order, so take LOGIT_TOL = GAP / 4 as that agreement. A logit error of at
+# most d moves the weight softmax(l)_j by at most 2 d w_j (one term from l_j,
+# one from the normaliser), hence the relative bound W_REL.
+LOGIT_TOL = GAP / 4
+W_REL = 2 * LOGIT_TOL
 
 SMALL = inputs.Dims(embed_dim=256, num_experts=16, expert_dim=192, hidden_dim=320)
 
@@ -85,7 +92,7 @@ def check_routing(ref_logits, ref_idx, ref_w, idx, w, k):
     s = -np.sort(-ref_logits, axis=1)[:, :k]
     order_clear = np.all(-np.diff(s, axis=1) > GAP, axis=1) & clear
     np.testing.assert_array_equal(idx[order_clear], ref_idx[order_clear])
-    np.testing.assert_allclose(w[order_clear], ref_w[order_clear], rtol=0, atol=W_TOL)
+    np.testing.assert_allclose(w[order_clear], ref_w[order_clear], rtol=W_REL, atol=1e-9)
     # every token: k distinct experts, weights sum to one and do not increase
     assert all(len(set(r)) == k for r in idx)
     np.testing.assert_allclose(w.sum(1), 1.0, atol=1e-5)
