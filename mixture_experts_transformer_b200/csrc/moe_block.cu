@@ -44,6 +44,10 @@ struct Layout {
 
 // Large batches (experts average >= 160 routed rows) use the paired gate|up GEMM.
 bool paired_gateup(const Dims& d) { return static_cast<long long>(d.T) * d.k >= 160LL * d.E; }
+// The paired down GEMM pays off later (measured: at ~256 rows per expert it is
+// slower, at ~1024 faster): its K = expert_dim is short, so a tile's single-
+// buffered accumulators drain often.
+bool paired_down(const Dims& d) { return static_cast<long long>(d.T) * d.k >= 512LL * d.E; }
 
 // Splits of the router's reduction: enough (token tile, split) CTAs for one
 // wave at one CTA per SM, at least two 64-wide slices per split.
@@ -149,6 +153,9 @@ moe_status device_state(DeviceState** out) {
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaFuncSetAttribute(grouped_gemm_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kGemmSmemBytes) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(grouped_gemm_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaFuncSetAttribute(fp4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
@@ -396,7 +403,8 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256, paired_gateup(d) ? 1 : 0);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256, paired_gateup(d) ? 1 : 0,
+                                     paired_down(d) ? 1 : 0);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
@@ -466,7 +474,9 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   const int grid_dn = std::min(s->sm_count, L.max_tiles_dn);
   {
   LaunchScope ls_(kKGemmDown, st);
-  const cudaError_t le_ = launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn);
+  const cudaError_t le_ =
+      paired_down(d) ? launch_k(grouped_gemm_kernel<false, true>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn)
+                     : launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn);
   MOE_TRY(ls_.done(le_));
   }
 
@@ -622,7 +632,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 0);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 0, 0);
     MOE_TRY(ls_.done(le_));
   }
   {

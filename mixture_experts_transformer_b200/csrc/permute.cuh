@@ -58,11 +58,11 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
                                                                   Tile* __restrict__ tiles_gu,
                                                                   Tile* __restrict__ tiles_dn,
                                                                   TileCounts* __restrict__ counts, int padded,
-                                                                  int dn_cols, int pair_gu) {
+                                                                  int dn_cols, int pair_gu, int pair_dn) {
   __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
-  __shared__ int s_ptoff[129];  // prefix of gate|up row-tile pairs per expert
+  __shared__ int s_ptoff[129];  // prefix of 128-row block pairs per expert (paired GEMM tiles)
   __shared__ int s_cnt[128];
   pdl_wait_then_release();
   const int e = threadIdx.x & 127;
@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     for (int b = 0; b < 128; b += 32) {
       const int v = s_cnt[b + lane];
       const int mv = (v + kBM - 1) / kBM;
-      const int pv = pair_gu ? (mv + 1) / 2 : mv;
+      const int pv = (mv + 1) / 2;
       int inc = v, minc = mv, pinc = pv;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -137,61 +137,47 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   }
   if (threadIdx.x == 0) off_out[E] = s_off[E];
 
-  // gate|up tiles take one 128-row block (pair_gu = 0) or two consecutive
-  // ones of the same expert and column tile (pair_gu = 1, the paired GEMM)
-  const int mstep = pair_gu ? 2 : 1;
+  // A tile takes one 128-row block, or (paired GEMM) two consecutive blocks of
+  // the same expert and column tile. Gate|up tiles are 128 output columns per
+  // projection, down tiles dn_cols wide.
   const int mt_sh = (T + kBM - 1) / kBM;
-  const int pt_sh = (mt_sh + mstep - 1) / mstep;
-  const int nt_gu_sh = (S + 127) / 128;
   const int nt_gu = (F + 127) / 128;
   const int nt_dn = (D + dn_cols - 1) / dn_cols;
-  const int n_sh_gu = nt_gu_sh * pt_sh;
-  const int n_sh_dn = nt_dn * mt_sh;
-  for (int i = threadIdx.x; i < n_sh_gu; i += kScanThreads) {
-    const int nt = i / pt_sh, m = (i % pt_sh) * mstep;
-    const int r1 = pair_gu ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
-    tiles_gu[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * 128, (m + 1) * kBM, r1, {0, 0}};
-  }
-  for (int i = threadIdx.x; i < n_sh_dn; i += kScanThreads) {
-    const int nt = i / mt_sh, m = i % mt_sh;
-    tiles_dn[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
-  }
-  // expert tiles, spread over all threads (one expert may own most of them):
-  // flat index f -> expert by binary search over the tile-offset prefix
-  const int n_e_gu = s_ptoff[E] * nt_gu;
-  for (int f = threadIdx.x; f < n_e_gu; f += kScanThreads) {
-    int lo = 0, hi = E - 1;  // largest ex with s_ptoff[ex] * nt_gu <= f
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_ptoff[mid] * nt_gu <= f) lo = mid; else hi = mid - 1;
+  auto emit = [&](Tile* tiles, int pair, int ncol_sh, int ncol, int cw) -> int {
+    const int mstep = pair ? 2 : 1;
+    const int* offs = pair ? s_ptoff : s_mtoff;
+    const int pt_sh = (mt_sh + mstep - 1) / mstep;
+    const int n_sh = ncol_sh * pt_sh;
+    for (int i = threadIdx.x; i < n_sh; i += kScanThreads) {
+      const int nt = i / pt_sh, m = (i % pt_sh) * mstep;
+      const int r1 = pair ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
+      tiles[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, {0, 0}};
     }
-    const int ex = lo;
-    const int ce = s_cnt[ex];
-    const int pt = s_ptoff[ex + 1] - s_ptoff[ex];
-    const int i = f - s_ptoff[ex] * nt_gu;
-    const int nt = i / pt, m = (i % pt) * mstep;
-    const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
-    const int r1 = pair_gu ? max(0, min(kBM, ce - (m + 1) * kBM)) : 0;
-    tiles_gu[n_sh_gu + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * 128, rb + (m + 1) * kBM, r1, {0, 0}};
-  }
-  const int n_e_dn = s_mtoff[E] * nt_dn;
-  for (int f = threadIdx.x; f < n_e_dn; f += kScanThreads) {
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_mtoff[mid] * nt_dn <= f) lo = mid; else hi = mid - 1;
+    // expert tiles, spread over all threads (one expert may own most of them):
+    // flat index f -> expert by binary search over the tile-offset prefix
+    const int n_e = offs[E] * ncol;
+    for (int f = threadIdx.x; f < n_e; f += kScanThreads) {
+      int lo = 0, hi = E - 1;  // largest ex with offs[ex] * ncol <= f
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offs[mid] * ncol <= f) lo = mid; else hi = mid - 1;
+      }
+      const int ex = lo;
+      const int ce = s_cnt[ex];
+      const int pt = offs[ex + 1] - offs[ex];
+      const int i = f - offs[ex] * ncol;
+      const int nt = i / pt, m = (i % pt) * mstep;
+      const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
+      const int r1 = pair ? max(0, min(kBM, ce - (m + 1) * kBM)) : 0;
+      tiles[n_sh + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * cw, rb + (m + 1) * kBM, r1, {0, 0}};
     }
-    const int ex = lo;
-    const int ce = s_cnt[ex];
-    const int mt = s_mtoff[ex + 1] - s_mtoff[ex];
-    const int i = f - s_mtoff[ex] * nt_dn;
-    const int nt = i / mt, m = i % mt;
-    const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
-    tiles_dn[n_sh_dn + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * dn_cols, 0, 0, {0, 0}};
-  }
+    return n_sh + n_e;
+  };
+  const int n_gu = emit(tiles_gu, pair_gu, (S + 127) / 128, nt_gu, 128);
+  const int n_dn = emit(tiles_dn, pair_dn, (D + dn_cols - 1) / dn_cols, nt_dn, dn_cols);
   if (threadIdx.x == 0) {
-    counts->gateup = n_sh_gu + s_ptoff[E] * nt_gu;
-    counts->down = n_sh_dn + s_mtoff[E] * nt_dn;
+    counts->gateup = n_gu;
+    counts->down = n_dn;
   }
 }
 
