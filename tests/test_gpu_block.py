@@ -101,10 +101,12 @@ def test_permute_bit_exact(T, skew):
 # -------------------------------------------------------------- the block
 
 
-@pytest.mark.parametrize("T,k", [(1, 4), (7, 4), (65, 4), (300, 4), (300, 1), (513, 8)])
+@pytest.mark.parametrize("T,k", [(1, 4), (7, 4), (65, 4), (300, 4), (300, 1), (513, 8), (1100, 8)])
 def test_block_small_dims(T, k):
     """Dims 256/16/192/320 put a 64-column tail tile on every GEMM; T spans
-    partial and multiple 128-row tiles."""
+    partial and multiple 128-row tiles. T*k = 4104 takes the paired gate|up
+    GEMM (>= 160 rows per expert on average), 8800 the paired down GEMM too
+    (>= 512)."""
     w = weights(SMALL, seed=1, std=0.05)
     dw = device_weights(SMALL, seed=1, std=0.05)
     x_bits = inputs.make_x(T, SMALL.embed_dim, seed=T)
