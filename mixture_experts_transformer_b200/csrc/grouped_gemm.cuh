@@ -47,7 +47,9 @@ constexpr int kBStageBytes = kMaxBChunks * kBChunkBytes;
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
 constexpr int kGemmThreads = 320;
-constexpr int kGemmSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kEpiWarps = 8;
+constexpr int kTileRing = 8;  // tile indices handed from the producer to the MMA and epilogue warps
+constexpr int kGemmSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 /*align*/ + 512 /*barriers, ring*/;
 
 // One 128-row work tile. pg = (problem << 16) | group.
 struct Tile {
@@ -78,6 +80,7 @@ struct GemmParams {
   int nprob;
   const Tile* tiles;
   const int32_t* num_tiles;
+  int32_t* next_tile;  // work counter, zero at launch: CTAs take tiles in list order as they free up
   uint32_t* err;
 };
 
@@ -102,8 +105,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* tile_full = drain + 1;
+  uint64_t* tile_empty = tile_full + kTileRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_empty + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* tile_ring = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -118,6 +124,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       mbar_init(&acc_empty[a], PAIRED ? 4 : 8);  // one arrival per epilogue warp draining it
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < kTileRing; ++r) {
+      mbar_init(&tile_full[r], 1);
+      mbar_init(&tile_empty[r], 1 + kEpiWarps);  // the MMA thread and every epilogue warp read each index
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -143,11 +153,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 
   if (warp == 0) {
     // -------------------------------------------------------- TMA producer
-    // The whole warp walks the tiles; lane 0 arms each stage's barrier and
-    // issues the loads.
+    // The whole warp walks the tiles; lane 0 takes the next tile index from
+    // the work counter, publishes it in the tile ring (-1 ends the work), arms
+    // each stage's barrier and issues the loads.
     int s = 0, issued = 0;
     uint32_t ph = 0;
-    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+    int rs = 0;
+    uint32_t rph = 0;
+    int ti = 0;
+    if (lane == 0) ti = atomicAdd(P.next_tile, 1);
+    ti = __shfl_sync(0xffffffffu, ti, 0);
+    while (true) {
+      int pub = 1;
+      if (lane == 0) {
+        pub = mbar_wait(&tile_empty[rs], rph ^ 1, abort_flag, P.err);
+        if (pub) {
+          tile_ring[rs] = ti < num_tiles ? ti : -1;
+          mbar_arrive(&tile_full[rs]);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, pub, 0)) break;
+      if (++rs == kTileRing) {
+        rs = 0;
+        rph ^= 1;
+      }
+      if (ti >= num_tiles) break;
+      int next = 0;
+      if (lane == 0) next = atomicAdd(P.next_tile, 1);  // its latency hides behind this tile's loads
       const Tile tile = P.tiles[ti];
       const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
       const bool bad_p = p >= P.nprob;
@@ -194,6 +226,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         }
       }
       if (!ok) break;
+      ti = __shfl_sync(0xffffffffu, next, 0);
     }
     __syncwarp();
     if (lane == 0 && *abort_flag) {
@@ -216,7 +249,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       int s = 0, acc = 0;
       uint32_t ph = 0, acc_ph = 0;
       bool any = false;
-      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      int rs = 0;
+      uint32_t rph = 0;
+      while (true) {
+        if (!mbar_wait(&tile_full[rs], rph, abort_flag, P.err)) break;
+        const int ti = tile_ring[rs];
+        mbar_arrive(&tile_empty[rs]);
+        if (++rs == kTileRing) {
+          rs = 0;
+          rph ^= 1;
+        }
+        if (ti < 0) break;
         const Tile tile = P.tiles[ti];
         const int p = tile.pg >> 16;
         if (p >= P.nprob) break;
@@ -282,7 +325,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     const int j_step = PAIRED ? 32 : 64;
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+    int rs = 0;
+    uint32_t rph = 0;
+    while (true) {
+      const bool got = mbar_wait(&tile_full[rs], rph, abort_flag, P.err);
+      int ti = got ? tile_ring[rs] : -1;
+      __syncwarp();
+      if (lane == 0 && got) mbar_arrive(&tile_empty[rs]);
+      if (++rs == kTileRing) {
+        rs = 0;
+        rph ^= 1;
+      }
+      ti = __shfl_sync(0xffffffffu, ti, 0);
+      if (ti < 0) break;
       const Tile tile = P.tiles[ti];
       const int p = tile.pg >> 16;
       if (p >= P.nprob) break;

@@ -430,7 +430,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(ws + L.hs);
   float* sbuf = reinterpret_cast<float*>(ws + L.s);
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
-  const TileCounts* counts = reinterpret_cast<const TileCounts*>(ws + L.counts);
+  TileCounts* counts = reinterpret_cast<TileCounts*>(ws + L.counts);
 
   MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
   MOE_TRY(enqueue_permute(d, L, ws, idx, p->x, cnt, off, row_of, token_of, st));
@@ -447,6 +447,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   gu.nprob = 2;
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
+  gu.next_tile = &counts->next_gateup;
   gu.err = s->err;
   const int grid_gu = std::min(s->sm_count, L.max_tiles_gu);
   {
@@ -470,6 +471,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   dn.nprob = 2;
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
+  dn.next_tile = &counts->next_down;
   dn.err = s->err;
   const int grid_dn = std::min(s->sm_count, L.max_tiles_dn);
   {
@@ -624,7 +626,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   int32_t* row_of = reinterpret_cast<int32_t*>(ws + L.row_of);
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(ws + L.masks);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
-  const TileCounts* counts = reinterpret_cast<const TileCounts*>(ws + L.counts);
+  TileCounts* counts = reinterpret_cast<TileCounts*>(ws + L.counts);
 
   MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
   {

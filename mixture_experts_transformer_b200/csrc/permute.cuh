@@ -25,6 +25,8 @@ constexpr int kScanSegs = kScanThreads / 128;
 struct TileCounts {
   int32_t gateup;
   int32_t down;
+  int32_t next_gateup;  // the GEMMs' work counters, cleared by the scan
+  int32_t next_down;
 };
 
 // Bitmasks of a given idx [T, k] (moe_permute's entry; the forward pass gets
@@ -178,6 +180,8 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   if (threadIdx.x == 0) {
     counts->gateup = n_gu;
     counts->down = n_dn;
+    counts->next_gateup = 0;
+    counts->next_down = 0;
   }
 }
 
