@@ -49,7 +49,9 @@ constexpr int kTmemCols = 512;
 constexpr int kGemmThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kTileRing = 8;  // tile indices handed from the producer to the MMA and epilogue warps
-constexpr int kGemmSmemBytes = kStages * (kAStageBytes + kBStageBytes) + 1024 /*align*/ + 512 /*barriers, ring*/;
+constexpr int kStageBytesTotal = kStages * (kAStageBytes + kBStageBytes);
+constexpr int kStgWarpBytes = 4096;  // epilogue staging: 32 rows x 128 B per warp
+constexpr int kGemmSmemBytes = kStageBytesTotal + kEpiWarps * kStgWarpBytes + 1024 /*align*/ + 512 /*barriers, ring*/;
 
 // One 128-row work tile. pg = (problem << 16) | group.
 struct Tile {
@@ -84,6 +86,44 @@ struct GemmParams {
   uint32_t* err;
 };
 
+// The epilogue holds one output row per thread (the TMEM lane layout). Rows
+// are passed through the warp's staging buffer so that the global stores are
+// whole 32-byte sectors of consecutive rows rather than 16-byte pieces of 32
+// different rows: each lane writes its row's 16-byte pieces with an XOR
+// swizzle (conflict-free), then the warp stores 16 bytes per lane in row
+// order. Rows at or past rows_valid are not stored.
+__device__ __forceinline__ void store_rows_bf16x32(uint8_t* stg, const uint32_t (&pk)[16], int lane,
+                                                   __nv_bfloat16* base, size_t ldo, int rows_valid) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    *reinterpret_cast<uint4*>(stg + lane * 64 + ((v ^ (lane & 3)) << 4)) =
+        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 32 + lane, row = idx >> 2, v = idx & 3;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 64 + ((v ^ (row & 3)) << 4));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 8) = val;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_rows_f32x32(uint8_t* stg, const uint32_t (&a)[32], int lane, float* base,
+                                                  size_t ldo, int rows_valid) {
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    *reinterpret_cast<uint4*>(stg + lane * 128 + ((v ^ (lane & 7)) << 4)) =
+        make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int idx = it * 32 + lane, row = idx >> 3, v = idx & 7;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((v ^ (row & 7)) << 4));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 4) = val;
+  }
+  __syncwarp();
+}
+
 template <bool GATEUP>
 __device__ __forceinline__ int tile_cols(const GemmProblem& pr, int n0) {
   const int cap = GATEUP ? 128 : 256;
@@ -100,7 +140,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kSt * kAS;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * (kAStageBytes + kBStageBytes));
+  uint8_t* sStg = smem + kStageBytesTotal;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + kEpiWarps * kStgWarpBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
@@ -320,7 +361,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     // ----------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter..+31
     const int half = (warp - 2) >> 2;  // unpaired: column chunks j = 32 * half + 64 c; PAIRED: the accumulator
-    const int r = quarter * 32 + lane;
     const int j_first = PAIRED ? 0 : 32 * half;
     const int j_step = PAIRED ? 32 : 64;
     int acc = 0;
@@ -351,11 +391,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const uint32_t tbase = tmem_base + a_id * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
       const int t_rows = (PAIRED && half) ? tile.rows1 : tile.rows;
       const int t_row0 = (PAIRED && half) ? tile.row1 : tile.row0;
-      const bool valid = r < t_rows;
-      const size_t grow = static_cast<size_t>(t_row0 + r);
+      const int rows_valid = t_rows - quarter * 32;  // of this warp's 32 rows
+      const size_t wrow = static_cast<size_t>(t_row0 + quarter * 32);
+      uint8_t* stg = sStg + (warp - 2) * kStgWarpBytes;
       if (!(PAIRED && half && t_rows <= 0)) {
       if (GATEUP) {
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo + tile.n0;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out) + wrow * pr.ldo + tile.n0;
         for (int j = j_first; j < wn; j += j_step) {
           uint32_t g[32], u[32];
           tmem_ld_32x32b_x32(tbase + j, g);
@@ -368,34 +409,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             const float h1 = gelu_tanh(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
             pk[i] = pack_bf16x2(h0, h1);
           }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + j);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          }
+          store_rows_bf16x32(stg, pk, lane, out + j, pr.ldo, rows_valid);
         }
       } else {
         for (int j = j_first; j < wn; j += j_step) {
           uint32_t a[32];
           tmem_ld_32x32b_x32(tbase + j, a);
           tmem_ld_wait();
-          if (valid) {
-            if (pr.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + grow * pr.ldo + tile.n0 + j);
+          if (pr.out_f32) {
+            store_rows_f32x32(stg, a, lane, reinterpret_cast<float*>(pr.out) + wrow * pr.ldo + tile.n0 + j, pr.ldo,
+                              rows_valid);
+          } else {
+            uint32_t pk[16];
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                dst[v] = make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                     __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo +
-                                                    tile.n0 + j);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * v]), __uint_as_float(a[8 * v + 1])),
-                                    pack_bf16x2(__uint_as_float(a[8 * v + 2]), __uint_as_float(a[8 * v + 3])),
-                                    pack_bf16x2(__uint_as_float(a[8 * v + 4]), __uint_as_float(a[8 * v + 5])),
-                                    pack_bf16x2(__uint_as_float(a[8 * v + 6]), __uint_as_float(a[8 * v + 7])));
-            }
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+            store_rows_bf16x32(stg, pk, lane, reinterpret_cast<__nv_bfloat16*>(pr.out) + wrow * pr.ldo + tile.n0 + j,
+                               pr.ldo, rows_valid);
           }
         }
       }
