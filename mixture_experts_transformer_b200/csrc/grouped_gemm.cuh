@@ -53,8 +53,9 @@ constexpr int kStageBytesTotal = kStages * (kAStageBytes + kBStageBytes);
 constexpr int kStgWarpBytes = 4096;  // epilogue staging: 32 rows x 128 B per warp
 constexpr int kGemmSmemBytes = kStageBytesTotal + kEpiWarps * kStgWarpBytes + 1024 /*align*/ + 512 /*barriers, ring*/;
 
-// One 128-row work tile. pg = (problem << 16) | group.
-struct Tile {
+// One 128-row work tile. pg = (problem << 16) | group. 16-byte aligned so a
+// tile moves as two vector accesses.
+struct __align__(16) Tile {
   int32_t pg;
   int32_t row0;   // first A row
   int32_t rows;   // rows of A that belong to this tile (1..128)

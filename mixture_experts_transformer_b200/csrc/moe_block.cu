@@ -54,7 +54,7 @@ bool paired_down(const Dims& d) { return static_cast<long long>(d.T) * d.k >= 51
 int router_splits(const Dims& d) {
   const int tiles = std::max(1, (d.T + kRouterTokens - 1) / kRouterTokens);
   int ns = kSmCountHint / tiles;
-  ns = std::min(ns, 22);
+  ns = std::min(ns, kMaxRouterSplits);
   ns = std::min(ns, d.D / (2 * kRouterBK));
   return std::max(ns, 1);
 }

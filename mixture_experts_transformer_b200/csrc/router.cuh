@@ -28,6 +28,7 @@ constexpr int kRouterBStage = 2 * kRouterBChunk;              // up to 128 exper
 constexpr int kRouterSmemBytes = kRouterStages * (kRouterAStage + kRouterBStage) + 1024 + 256;
 constexpr int kMaskTokens = 32;     // tokens per bitmask word
 constexpr int kTopkWarps = 4;       // one warp per token
+constexpr int kMaxRouterSplits = 22; // splits of the router's reduction (at most)
 
 struct RouterParams {
   CUtensorMap tmX;  // x [T, D] bf16, box 64 (K) x 128 (tokens), 128-byte swizzle
