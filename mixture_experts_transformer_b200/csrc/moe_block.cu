@@ -13,6 +13,7 @@
 
 #include "moe_block.h"
 #include "grouped_gemm.cuh"
+#include "grouped_gemm_pair.cuh"
 #include "permute.cuh"
 #include "router.cuh"
 #include "nvfp4.cuh"
@@ -128,8 +129,18 @@ struct DeviceState {
   uint32_t* err = nullptr;
   void* ws = nullptr;
   size_t ws_bytes = 0;
+  int pair_clusters_dn = 0;  // SM-pair clusters of the pair down GEMM that fit on the device at once
 };
 DeviceState g_dev[kMaxDevices];
+
+// Large batches run the down GEMM on SM pairs (tcgen05 cta_group::2) when its
+// column tiles split into whole 64-column chunks per CTA. (The gate|up GEMM
+// stays on single SMs: measured slower on pairs, whose M = 256 MMA runs in
+// full for an expert's odd last row block over the long K = embed_dim.)
+bool pair_sm(const Dims& d, const DeviceState* s) {
+  return static_cast<long long>(d.T) * d.k >= 160LL * d.E && d.D % 128 == 0 && s->pair_clusters_dn > 0;
+}
+
 
 moe_status device_state(DeviceState** out) {
   int dev = 0;
@@ -158,6 +169,17 @@ moe_status device_state(DeviceState** out) {
       if (cudaFuncSetAttribute(grouped_gemm_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kGemmSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kP2SmemBytes) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (s.sm_count / 2));
+        cfg.blockDim = dim3(kGemmThreads);
+        cfg.dynamicSmemBytes = kP2SmemBytes;
+        if (cudaOccupancyMaxActiveClusters(&s.pair_clusters_dn, grouped_gemm_pair_kernel<false>, &cfg) != cudaSuccess)
+          return MOE_ERR_CUDA;
+      }
       if (cudaFuncSetAttribute(fp4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
           cudaSuccess)
         return MOE_ERR_CUDA;
@@ -398,13 +420,16 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
                            int32_t* cnt, int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st) {
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(ws + L.masks);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  const bool pairs = pair_sm(d, s);
   {
     LaunchScope ls_(kKRouteScan, st);
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256, paired_gateup(d) ? 1 : 0,
-                                     paired_down(d) ? 1 : 0);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256,
+                                     paired_gateup(d) ? 1 : 0, (pairs || paired_down(d)) ? 1 : 0);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
@@ -477,8 +502,9 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   {
   LaunchScope ls_(kKGemmDown, st);
   const cudaError_t le_ =
-      paired_down(d) ? launch_k(grouped_gemm_kernel<false, true>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn)
-                     : launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn);
+      pair_sm(d, s) ? launch_k(grouped_gemm_pair_kernel<false>, 2 * s->pair_clusters_dn, kGemmThreads, kP2SmemBytes, st, dn)
+      : paired_down(d) ? launch_k(grouped_gemm_kernel<false, true>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn)
+                       : launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn);
   MOE_TRY(ls_.done(le_));
   }
 
