@@ -87,44 +87,6 @@ struct GemmParams {
   uint32_t* err;
 };
 
-// The epilogue holds one output row per thread (the TMEM lane layout). Rows
-// are passed through the warp's staging buffer so that the global stores are
-// whole 32-byte sectors of consecutive rows rather than 16-byte pieces of 32
-// different rows: each lane writes its row's 16-byte pieces with an XOR
-// swizzle (conflict-free), then the warp stores 16 bytes per lane in row
-// order. Rows at or past rows_valid are not stored.
-__device__ __forceinline__ void store_rows_bf16x32(uint8_t* stg, const uint32_t (&pk)[16], int lane,
-                                                   __nv_bfloat16* base, size_t ldo, int rows_valid) {
-#pragma unroll
-  for (int v = 0; v < 4; ++v)
-    *reinterpret_cast<uint4*>(stg + lane * 64 + ((v ^ (lane & 3)) << 4)) =
-        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-  __syncwarp();
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int idx = it * 32 + lane, row = idx >> 2, v = idx & 3;
-    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 64 + ((v ^ (row & 3)) << 4));
-    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 8) = val;
-  }
-  __syncwarp();
-}
-
-__device__ __forceinline__ void store_rows_f32x32(uint8_t* stg, const uint32_t (&a)[32], int lane, float* base,
-                                                  size_t ldo, int rows_valid) {
-#pragma unroll
-  for (int v = 0; v < 8; ++v)
-    *reinterpret_cast<uint4*>(stg + lane * 128 + ((v ^ (lane & 7)) << 4)) =
-        make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
-  __syncwarp();
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int idx = it * 32 + lane, row = idx >> 3, v = idx & 7;
-    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((v ^ (row & 7)) << 4));
-    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 4) = val;
-  }
-  __syncwarp();
-}
-
 template <bool GATEUP>
 __device__ __forceinline__ int tile_cols(const GemmProblem& pr, int n0) {
   const int cap = GATEUP ? 128 : 256;

@@ -222,7 +222,8 @@ constexpr int kF4SfBytes = 4 * 512;              // 4 atoms (4 x 64 K) of one 12
 constexpr int kF4Stages = 4;
 constexpr int kF4SfSlots = 16;                   // TMEM scale slots (ring over 64-K steps)
 constexpr int kF4Threads = 320;                  // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
-constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 1024 + 256;
+constexpr int kF4StgWarpBytes = 1024;            // epilogue staging per warp (32 rows x 32 B)
+constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 8 * kF4StgWarpBytes + 1024 + 256;
 
 struct Fp4Problem {
   int K;          // multiple of 64
@@ -316,7 +317,8 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
   uint8_t* sB = sA + kF4Stages * kF4ABytes;
   uint8_t* sSfA = sB + kF4Stages * kF4BBytes;
   uint8_t* sSfB = sSfA + kF4Stages * kF4SfBytes;  // per stage: block 0 atoms, then block 1 atoms
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSfB + kF4Stages * 2 * kF4SfBytes);
+  uint8_t* sStg = sSfB + kF4Stages * 2 * kF4SfBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStg + 8 * kF4StgWarpBytes);
   uint64_t* empty = full + kF4Stages;
   constexpr int kAccStages = 1;
   constexpr uint32_t kAccStride = 256;
@@ -439,6 +441,7 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
       uint32_t ph = 0, acc_ph = 0;
       bool any = false;
       const uint32_t idesc = idesc_nvf4_m128(128);
+      const uint32_t idesc256 = idesc_nvf4_m128(256);
       for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
         const Tile tile = P.tiles[ti];
         const int p = tile.pg >> 16;
@@ -475,11 +478,10 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
             const uint64_t ad = sdesc_sw128(a_addr + i * 32, 16, 1024);
             const uint64_t bd0 = sdesc_sw128(b_addr + i * 32, 16, 1024);
             const uint32_t accum = (ks | i) != 0;
-            umma_nvf4(d_tmem, ad, bd0, idesc, cols, cols + 4, accum);
-            if (two_b) {
-              const uint64_t bd1 = sdesc_sw128(b_addr + kF4BBytes / 2 + i * 32, 16, 1024);
-              umma_nvf4(d_tmem + 128, ad, bd1, idesc, cols, cols + 8, accum);
-            }
+            // both B blocks (gate | up, or 256 output columns) are consecutive
+            // 128-row halves of the stage and their scale atoms sit at cols + 4
+            // and cols + 8, which is the N = 256 layout: one MMA covers both
+            umma_nvf4(d_tmem, ad, bd0, two_b ? idesc256 : idesc, cols, cols + 4, accum);
           }
           slot = (slot + nks) % kF4SfSlots;
           any = true;
@@ -569,30 +571,32 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
             pr.out_sf[sf_offset(grow, c16 + 1, pr.N / 64)] = static_cast<uint8_t>(sc[1]);
           }
         }
-      } else if (valid) {
+      } else {
+        // staged through the warp's buffer: whole-sector stores in row order
         const float alpha = 1.0f / (pr.ga * pr.gb0[g]);
+        uint8_t* stg = sStg + (warp - 2) * kF4StgWarpBytes;
+        const int rows_valid = tile.rows - quarter * 32;
+        const size_t wrow = static_cast<size_t>(tile.row0 + quarter * 32);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int j = half * 32 + 64 * c;
           if (j >= wn) continue;
-          const uint32_t* a = acc[c];
+          uint32_t* a = acc[c];
           if (pr.out_f32) {
-            float4* dst =
-                reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(a[4 * v]) * alpha, __uint_as_float(a[4 * v + 1]) * alpha,
-                                   __uint_as_float(a[4 * v + 2]) * alpha, __uint_as_float(a[4 * v + 3]) * alpha);
+            for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+            uint8_t* base = reinterpret_cast<uint8_t*>(reinterpret_cast<float*>(pr.out) + wrow * pr.ldo + tile.n0 + j);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) store_rows_32B(stg, a + 8 * q, lane, base + 32 * q, pr.ldo * 4, rows_valid);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) +
-                                                  static_cast<size_t>(grow) * pr.ldo + tile.n0 + j);
+            uint32_t pk[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(
-                  pack_bf16x2(__uint_as_float(a[8 * v]) * alpha, __uint_as_float(a[8 * v + 1]) * alpha),
-                  pack_bf16x2(__uint_as_float(a[8 * v + 2]) * alpha, __uint_as_float(a[8 * v + 3]) * alpha),
-                  pack_bf16x2(__uint_as_float(a[8 * v + 4]) * alpha, __uint_as_float(a[8 * v + 5]) * alpha),
-                  pack_bf16x2(__uint_as_float(a[8 * v + 6]) * alpha, __uint_as_float(a[8 * v + 7]) * alpha));
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * alpha, __uint_as_float(a[2 * i + 1]) * alpha);
+            uint8_t* base =
+                reinterpret_cast<uint8_t*>(reinterpret_cast<__nv_bfloat16*>(pr.out) + wrow * pr.ldo + tile.n0 + j);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) store_rows_32B(stg, pk + 8 * q, lane, base + 32 * q, pr.ldo * 2, rows_valid);
           }
         }
       }

@@ -333,6 +333,64 @@ __host__ __device__ constexpr uint32_t idesc_bf16_m256(int n, int b_mn_major) {
          (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
+// ------------------------------------------------------- epilogue stores
+
+// The epilogue holds one output row per thread (the TMEM lane layout). Rows
+// are passed through the warp's staging buffer so that the global stores are
+// whole 32-byte sectors of consecutive rows rather than 16-byte pieces of 32
+// different rows: each lane writes its row's 16-byte pieces with an XOR
+// swizzle (conflict-free), then the warp stores 16 bytes per lane in row
+// order. Rows at or past rows_valid are not stored.
+__device__ __forceinline__ void store_rows_bf16x32(uint8_t* stg, const uint32_t (&pk)[16], int lane,
+                                                   __nv_bfloat16* base, size_t ldo, int rows_valid) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    *reinterpret_cast<uint4*>(stg + lane * 64 + ((v ^ (lane & 3)) << 4)) =
+        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 32 + lane, row = idx >> 2, v = idx & 3;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 64 + ((v ^ (row & 3)) << 4));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 8) = val;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_rows_f32x32(uint8_t* stg, const uint32_t (&a)[32], int lane, float* base,
+                                                  size_t ldo, int rows_valid) {
+#pragma unroll
+  for (int v = 0; v < 8; ++v)
+    *reinterpret_cast<uint4*>(stg + lane * 128 + ((v ^ (lane & 7)) << 4)) =
+        make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int idx = it * 32 + lane, row = idx >> 3, v = idx & 7;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 128 + ((v ^ (row & 7)) << 4));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 4) = val;
+  }
+  __syncwarp();
+}
+
+// The same through a 1 KB buffer: 32 bytes of each of the warp's 32 rows (this
+// lane's row in w), one whole sector per row.
+__device__ __forceinline__ void store_rows_32B(uint8_t* stg, const uint32_t* w, int lane, uint8_t* base, size_t pitch,
+                                               int rows_valid) {
+#pragma unroll
+  for (int v = 0; v < 2; ++v)
+    *reinterpret_cast<uint4*>(stg + lane * 32 + ((v ^ ((lane >> 2) & 1)) << 4)) =
+        make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 2; ++it) {
+    const int idx = it * 32 + lane, row = idx >> 1, v = idx & 1;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + row * 32 + ((v ^ ((row >> 2) & 1)) << 4));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * pitch + v * 16) = val;
+  }
+  __syncwarp();
+}
+
 // ------------------------------------------------------------- numerics
 
 __device__ __forceinline__ float tanh_approx(float x) {
