@@ -664,8 +664,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     MOE_TRY(ls_.done(le_));
   }
   {
-    const long long R = static_cast<long long>(d.T) * d.k;
-    const int blocks = static_cast<int>(std::min<long long>((R + 7) / 8, 148LL * 64));
+    const int blocks = static_cast<int>(std::min<long long>((d.T + 7) / 8, 148LL * 64));  // a warp per token
     LaunchScope ls_(kKScatterFp4, st);
     const cudaError_t le_ = launch_k(route_scatter_fp4_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E,
                                      d.D, static_cast<const __nv_bfloat16*>(p->x), p->g_x, row_of,

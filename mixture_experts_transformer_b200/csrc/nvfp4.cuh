@@ -176,40 +176,60 @@ __global__ void act_quant_kernel(const __nv_bfloat16* __restrict__ x, int rows, 
   }
 }
 
-// The NVFP4 block's scatter: one warp per (token, slot); its routed row in the
-// 128-padded expert-major row space comes from the bitmasks, the warp
-// quantises x[t] into that row (codes + scales) and, for slot 0, also into the
-// token-order buffer the shared MLP reads.
+// The NVFP4 block's scatter: one warp per token. The warp finds the routed
+// row of each of the token's k slots in the 128-padded expert-major row space
+// (from the bitmasks), quantises x[t] ONCE - each lane whole 64-element blocks,
+// i.e. 4 groups of 16: 32 bytes of codes and 4 scale bytes, which are one
+// aligned word of the scale atom - and writes the result to the token-order
+// buffer (the shared MLP's input) and to each routed row.
 __global__ void __launch_bounds__(256) route_scatter_fp4_kernel(
     const int32_t* __restrict__ idx, const uint32_t* __restrict__ masks, const int32_t* __restrict__ base, int T,
     int k, int E, int D, const __nv_bfloat16* __restrict__ x, float g_x, int32_t* __restrict__ row_of,
     uint8_t* __restrict__ xq_perm, uint8_t* __restrict__ xsf_perm, uint8_t* __restrict__ xq_tok,
     uint8_t* __restrict__ xsf_tok) {
+  __shared__ int s_rows[8][128];  // k <= num_experts <= 128
   pdl_wait_then_release();
-  const int lane = threadIdx.x & 31;
-  const long long R = static_cast<long long>(T) * k;
-  for (long long a = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); a < R;
-       a += static_cast<long long>(gridDim.x) * 8) {
-    const int t = static_cast<int>(a / k);
-    const int j = static_cast<int>(a % k);
-    const int e = __ldg(idx + a);
-    if (e < 0 || e >= E) continue;
-    const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
-    const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
-    const int row = __ldg(base + cw) + __popc(below);
-    if (lane == 0) row_of[a] = row;
-    for (int c = lane; c < D / 16; c += 32) {
-      float v[16];
-      load16_bf16(x + static_cast<size_t>(t) * D + c * 16, v);
-      uint2 codes;
-      const uint32_t sc = nvfp4_group(v, g_x, &codes);
-      *reinterpret_cast<uint2*>(xq_perm + static_cast<size_t>(row) * (D / 2) + c * 8) = codes;
-      xsf_perm[sf_offset(row, c, D / 64)] = static_cast<uint8_t>(sc);
-      if (j == 0) {
-        *reinterpret_cast<uint2*>(xq_tok + static_cast<size_t>(t) * (D / 2) + c * 8) = codes;
-        xsf_tok[sf_offset(t, c, D / 64)] = static_cast<uint8_t>(sc);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int k64 = D / 64;
+  for (int t = blockIdx.x * 8 + wid; t < T; t += gridDim.x * 8) {
+    for (int j = lane; j < k; j += 32) {
+      const long long a = static_cast<long long>(t) * k + j;
+      const int e = __ldg(idx + a);
+      int row = -1;
+      if (e >= 0 && e < E) {
+        const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
+        const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
+        row = __ldg(base + cw) + __popc(below);
+        row_of[a] = row;
+      }
+      s_rows[wid][j] = row;
+    }
+    __syncwarp();
+    for (int b = lane; b < k64; b += 32) {
+      uint2 codes[4];
+      uint32_t scw = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[16];
+        load16_bf16(x + static_cast<size_t>(t) * D + b * 64 + q * 16, v);
+        scw |= (nvfp4_group(v, g_x, &codes[q]) & 0xFFu) << (8 * q);
+      }
+      const uint4 c0 = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+      const uint4 c1 = make_uint4(codes[2].x, codes[2].y, codes[3].x, codes[3].y);
+      uint4* qt = reinterpret_cast<uint4*>(xq_tok + static_cast<size_t>(t) * (D / 2) + b * 32);
+      qt[0] = c0;
+      qt[1] = c1;
+      *reinterpret_cast<uint32_t*>(xsf_tok + sf_offset(t, 4 * b, k64)) = scw;
+      for (int j = 0; j < k; ++j) {
+        const int row = s_rows[wid][j];
+        if (row < 0) continue;
+        uint4* qp = reinterpret_cast<uint4*>(xq_perm + static_cast<size_t>(row) * (D / 2) + b * 32);
+        qp[0] = c0;
+        qp[1] = c1;
+        *reinterpret_cast<uint32_t*>(xsf_perm + sf_offset(row, 4 * b, k64)) = scw;
       }
     }
+    __syncwarp();
   }
 }
 
