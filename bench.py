@@ -78,6 +78,8 @@ def parse():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sandwich", action="store_true",
+                    help="bf16 workloads: time the block with the pre/post-FFN RMSNorm sandwich and the residual add")
     ap.add_argument("--layers", type=int, default=None, help="nvfp4_stack depth (default 30)")
     return ap.parse_args()
 
@@ -295,10 +297,19 @@ def run_ours(args, world, rank, local):
     out = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
     ws, _ = block.workspace_for(inputs.GEMMA4_26B_A4B, T)
     stream = torch.cuda.current_stream()
-    p = B.make_params(T, x, *dw.args(), out, router_bias=bias, workspace=ws)
+    sandwich = {}
+    if args.sandwich:
+        # learned scales of the pre- and post-FFN RMSNorm, seeded U(0.5, 1.5)
+        gs = torch.Generator(device="cuda").manual_seed(9)
+        sandwich = {
+            "norm_pre": torch.empty(D, device="cuda").uniform_(0.5, 1.5, generator=gs).to(torch.bfloat16),
+            "norm_post": torch.empty(D, device="cuda").uniform_(0.5, 1.5, generator=gs).to(torch.bfloat16),
+            "residual": True,
+        }
+    p = B.make_params(T, x, *dw.args(), out, router_bias=bias, workspace=ws, **sandwich)
 
     # routing statistics of this batch (outside the timed region)
-    dbg = block.forward(dw, x, router_bias=bias, debug=True, workspace=ws)
+    dbg = block.forward(dw, x, router_bias=bias, debug=True, workspace=ws, **sandwich)
     torch.cuda.synchronize()
     cnt = dbg.cnt.cpu().numpy()
     touched = int((cnt > 0).sum())
@@ -399,12 +410,13 @@ def run_ours(args, world, rank, local):
         "dtype": "bf16",
         "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, x ~ N(0,1)",
         "config": {
-            "workload": wl["desc"],
+            "workload": wl["desc"] + (", with the pre/post-FFN RMSNorm sandwich and residual" if args.sandwich else ""),
             "tokens_per_gpu": T,
             "global_batch": T * world,
             "parallelism": f"replicas{world}" if world > 1 else "single",
             "l2": "inputs larger than L2 (1.5 GB of expert weights per step)",
             "router_bias": "zipf(1.1)" if wl["bias"] else None,
+            "sandwich": bool(args.sandwich),
         },
         "roofline": {
             "bound": wl["bound"],
@@ -431,7 +443,7 @@ def run_ours(args, world, rank, local):
         "clocks": clocks.report(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(dw, x, bias, T, budget_s=12.0)
+        res["cpu_baseline"] = cpu_baseline(dw, x, bias, T, budget_s=12.0, sandwich=sandwich)
     return res
 
 
@@ -654,9 +666,10 @@ def _oracle_cores():
         return os.cpu_count()
 
 
-def cpu_baseline(dw, x, bias, T, budget_s=12.0, sample_tokens=None):
+def cpu_baseline(dw, x, bias, T, budget_s=12.0, sample_tokens=None, sandwich=None):
     """The oracle as it stands, on a bounded sample of the same workload."""
     from oracle import moe_oracle as mo
+    from oracle import sandwich as sw
 
     wh = _host_weights(dw)
     xb = x.cpu().view(__import__("torch").int16).numpy().view(np.uint16)
@@ -664,8 +677,14 @@ def cpu_baseline(dw, x, bias, T, budget_s=12.0, sample_tokens=None):
     n = min(T, sample_tokens or 64)
     xs = xb[:n]
     done, t0 = 0, time.perf_counter()
+    args_w = (wh.w_router, wh.wg, wh.wu, wh.wd, wh.sg, wh.su, wh.sd)
+    if sandwich:
+        g_pre, g_post = (sandwich[k].float().cpu().numpy() for k in ("norm_pre", "norm_post"))
     while True:
-        mo.moe_block(xs, wh.w_router, wh.wg, wh.wu, wh.wd, wh.sg, wh.su, wh.sd, top_k=K_TOP, bias=b)
+        if sandwich:
+            sw.sandwich_block(xs, *args_w, g_pre, g_post, top_k=K_TOP, bias=b)
+        else:
+            mo.moe_block(xs, *args_w, top_k=K_TOP, bias=b)
         done += n
         if time.perf_counter() - t0 > budget_s or done >= 64 * n:
             break
@@ -694,11 +713,20 @@ def run_reference(args, world, rank):
     n = min(T, 8)
     x = inputs.make_x(n)
     bias = inputs.zipf_router_bias() if wl["bias"] else None
+    args_w = (w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd)
+    if args.sandwich:
+        from oracle import sandwich as sw
+
+        rng = np.random.default_rng(9)
+        g_pre, g_post = rng.uniform(0.5, 1.5, D), rng.uniform(0.5, 1.5, D)
+        step = lambda: sw.sandwich_block(x, *args_w, g_pre, g_post, bias=bias)  # noqa: E731
+    else:
+        step = lambda: mo.moe_block(x, *args_w, bias=bias)  # noqa: E731
     for _ in range(args.warmup):
-        mo.moe_block(x, w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd, bias=bias)
+        step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        mo.moe_block(x, w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd, bias=bias)
+        step()
     el = time.perf_counter() - t0
     v = n * args.steps / el
     cores = _oracle_cores()
@@ -716,7 +744,13 @@ def run_reference(args, world, rank):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, x ~ N(0,1)",
-        "config": {"workload": wl["desc"], "tokens_per_gpu": T, "global_batch": T * world, "parallelism": "single"},
+        "config": {
+            "workload": wl["desc"] + (", with the pre/post-FFN RMSNorm sandwich and residual" if args.sandwich else ""),
+            "tokens_per_gpu": T,
+            "global_batch": T * world,
+            "parallelism": "single",
+            "sandwich": bool(args.sandwich),
+        },
         "cpu_baseline": {
             "value": v,
             "unit": "tokens/s",

@@ -91,6 +91,17 @@ typedef enum {
  *   out_f32 [T, embed_dim] fp32: the pre-rounding output (out == RNE(out_f32));
  *   idx_out [T, top_k] int32, w_out [T, top_k] fp32: the routing used;
  *   cnt_out [num_experts] int32: tokens per expert.
+ *
+ * The normalisation sandwich around the block (model card: RMSNorm layers,
+ * "sandwich" = pre and post, epsilon 1e-06), each part optional:
+ *   norm_pre  [embed_dim] bf16: the block computes on
+ *             x_n = RNE_bf16(norm_pre * x / sqrt(mean(x^2) + 1e-6)) (router,
+ *             experts and shared MLP all read x_n; kept in the workspace);
+ *   norm_post [embed_dim] bf16: the block output f becomes
+ *             norm_post * f / sqrt(mean(f^2) + 1e-6), in fp32;
+ *   residual  nonzero: out = RNE(x + that), the raw input x added in fp32.
+ * With norm_post or residual, embed_dim must be <= 4096. out_f32 then holds
+ * the final pre-rounding value.
  */
 typedef struct moe_params {
   int T;
@@ -115,6 +126,9 @@ typedef struct moe_params {
   int32_t* cnt_out;
   void* workspace;
   size_t workspace_bytes;
+  const void* norm_pre;
+  const void* norm_post;
+  int residual;
 } moe_params;
 
 /*
@@ -129,11 +143,13 @@ typedef struct moe_params {
  *   idx [T, top_k] int32, w [T, top_k] fp32, cnt [E] int32, off [E + 1] int32,
  *   row_of [T, top_k] int32 (routed row of each (token, slot)),
  *   token_of [R] int32 (token of each routed row)
+ *   x_norm [T, embed_dim] bf16   - the pre-normed block input (with norm_pre)
  */
 typedef struct moe_ws_layout {
   size_t total_bytes;
   size_t x_perm, h, y, hs, s;
   size_t idx, w, cnt, off, row_of, token_of;
+  size_t x_norm;
 } moe_ws_layout;
 
 /* Bytes of workspace a call with these params needs (T, top_k and dims are read). */

@@ -50,13 +50,17 @@ class MoeParams(ctypes.Structure):
         ("cnt_out", _vp),
         ("workspace", _vp),
         ("workspace_bytes", ctypes.c_size_t),
+        ("norm_pre", _vp),
+        ("norm_post", _vp),
+        ("residual", ctypes.c_int),
     ]
 
 
 class MoeWsLayout(ctypes.Structure):
     _fields_ = [
         (name, ctypes.c_size_t)
-        for name in ("total_bytes", "x_perm", "h", "y", "hs", "s", "idx", "w", "cnt", "off", "row_of", "token_of")
+        for name in ("total_bytes", "x_perm", "h", "y", "hs", "s", "idx", "w", "cnt", "off", "row_of", "token_of",
+                     "x_norm")
     ]
 
 
@@ -150,6 +154,9 @@ def make_params(
     cnt_out=None,
     workspace=None,
     workspace_bytes: int = 0,
+    norm_pre=None,
+    norm_post=None,
+    residual: bool = False,
 ) -> MoeParams:
     p = MoeParams()
     p.T = T
@@ -177,8 +184,11 @@ def make_params(
         ("w_out", w_out),
         ("cnt_out", cnt_out),
         ("workspace", workspace),
+        ("norm_pre", norm_pre),
+        ("norm_post", norm_post),
     ):
         setattr(p, name, ptr(val))
+    p.residual = 1 if residual else 0
     if workspace is not None and not workspace_bytes:
         workspace_bytes = workspace.numel() * workspace.element_size()
     p.workspace_bytes = workspace_bytes

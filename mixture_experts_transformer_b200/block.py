@@ -60,8 +60,13 @@ def forward(
     workspace: torch.Tensor | None = None,
     out: torch.Tensor | None = None,
     stream=None,
+    norm_pre: torch.Tensor | None = None,
+    norm_post: torch.Tensor | None = None,
+    residual: bool = False,
 ) -> BlockResult:
-    """Run one block; with debug=True also return out_f32, the routing and the counts."""
+    """Run one block; with debug=True also return out_f32, the routing and the counts.
+    norm_pre / norm_post (bf16 [embed_dim]) and residual add the normalisation
+    sandwich: out = x + norm_post-RMSNorm(block(norm_pre-RMSNorm(x)))."""
     T = x.shape[0]
     dev = x.device
     if out is None:
@@ -85,6 +90,9 @@ def forward(
         w_out=res.w,
         cnt_out=res.cnt,
         workspace=workspace,
+        norm_pre=norm_pre,
+        norm_post=norm_post,
+        residual=residual,
     )
     B.check(B.moe_block_forward_ex(p, stream), "moe_block_forward_ex")
     return res

@@ -14,6 +14,7 @@
 #include "moe_block.h"
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
+#include "norm.cuh"
 #include "permute.cuh"
 #include "router.cuh"
 #include "nvfp4.cuh"
@@ -39,7 +40,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Layout {
   size_t total;
   size_t partial, idx, w, masks, base, cnt, off, row_of, token_of, tiles_gu, tiles_dn, counts;
-  size_t x_perm, h, y, hs, s;
+  size_t x_perm, h, y, hs, s, x_norm;
   int nsplit, nchunks, max_tiles_gu, max_tiles_dn;
 };
 
@@ -92,6 +93,7 @@ Layout make_layout(const Dims& d) {
   L.y = take(R * d.D * 2);
   L.hs = take(T * d.S * 2);
   L.s = take(T * d.D * 4);
+  L.x_norm = take(T * d.D * 2);
   L.total = o;
   return L;
 }
@@ -275,6 +277,7 @@ enum KernelId : int {
   kKFp4Down,
   kKCombineNorm,
   kKAmax,
+  kKPreNorm,
   kKCount
 };
 const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "build_masks", "route_scan",
@@ -282,7 +285,7 @@ const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "buil
                                            "grouped_gemm_down", "combine", "timeout_probe",
                                            "nvfp4_weight_amax", "nvfp4_tensor_scale", "nvfp4_weight_quant",
                                            "nvfp4_act_quant", "route_scatter_fp4", "fp4_gemm_gateup",
-                                           "fp4_gemm_down", "combine_norm", "amax"};
+                                           "fp4_gemm_down", "combine_norm", "amax", "rms_norm_pre"};
 
 struct ProfRecord {
   int id;
@@ -370,6 +373,8 @@ moe_status check_block_args(const moe_params* p, Dims* d) {
   const uintptr_t xb = reinterpret_cast<uintptr_t>(p->x), ob = reinterpret_cast<uintptr_t>(p->out);
   const uintptr_t bytes = static_cast<uintptr_t>(d->T) * d->D * 2;
   if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
+  if ((p->norm_pre && !aligned16(p->norm_pre)) || (p->norm_post && !aligned16(p->norm_post))) return MOE_ERR_ALIGNMENT;
+  if ((p->norm_post || p->residual) && d->D > kCombThreads * kCombVec * 8) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -457,14 +462,25 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
   TileCounts* counts = reinterpret_cast<TileCounts*>(ws + L.counts);
 
-  MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
-  MOE_TRY(enqueue_permute(d, L, ws, idx, p->x, cnt, off, row_of, token_of, st));
+  // the block's input: x, or its pre-FFN RMSNorm (bf16, in the workspace)
+  const void* xin = p->x;
+  if (p->norm_pre) {
+    __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + L.x_norm);
+    LaunchScope ls_(kKPreNorm, st);
+    const int blocks = static_cast<int>(std::min<long long>((d.T + kNormWarps - 1) / kNormWarps, 148LL * 16));
+    MOE_TRY(ls_.done(launch_k(rms_norm_rows_kernel, blocks, kNormWarps * 32, 0, st,
+                              static_cast<const __nv_bfloat16*>(p->x),
+                              static_cast<const __nv_bfloat16*>(p->norm_pre), d.T, d.D, xn)));
+    xin = xn;
+  }
+  MOE_TRY(enqueue_route(d, L, ws, xin, p->w_router, p->router_bias, idx, w, st));
+  MOE_TRY(enqueue_permute(d, L, ws, idx, xin, cnt, off, row_of, token_of, st));
 
   // gate|up: experts (problem 0) and shared MLP (problem 1)
   GemmParams gu;
   std::memset(&gu, 0, sizeof(gu));
   bool ok = map_2d(&gu.tmA[0], x_perm, R, d.D, kBM) && map_3d(&gu.tmB0[0], p->wg, d.E, d.D, d.F) &&
-            map_3d(&gu.tmB1[0], p->wu, d.E, d.D, d.F) && map_2d(&gu.tmA[1], p->x, d.T, d.D, kBM) &&
+            map_3d(&gu.tmB1[0], p->wu, d.E, d.D, d.F) && map_2d(&gu.tmA[1], xin, d.T, d.D, kBM) &&
             map_3d(&gu.tmB0[1], p->sg, 1, d.D, d.S) && map_3d(&gu.tmB1[1], p->su, 1, d.D, d.S);
   if (!ok) return MOE_ERR_CUDA;
   gu.prob[0] = GemmProblem{d.D, d.F, d.E, static_cast<int>(R), h, d.F, 0};
@@ -508,7 +524,14 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   MOE_TRY(ls_.done(le_));
   }
 
-  {
+  if (p->norm_post || p->residual) {
+    // the post-FFN norm and / or the residual need a token's whole row: one CTA per token
+    LaunchScope ls_(kKCombineNorm, st);
+    MOE_TRY(ls_.done(launch_k(combine_norm_kernel, d.T, kCombThreads, 0, st, sbuf, y, row_of, w, d.T, d.k, d.D,
+                              p->norm_post ? 1 : 0, static_cast<const __nv_bfloat16*>(p->norm_post),
+                              p->residual ? static_cast<const __nv_bfloat16*>(p->x) : nullptr,
+                              static_cast<__nv_bfloat16*>(p->out), p->out_f32)));
+  } else {
   LaunchScope ls_(kKCombine, st);
   const int dsplit = std::max(1, std::min(4, (2 * s->sm_count) / std::max(1, d.T)));
   const cudaError_t le_ = launch_k(combine_kernel, dim3(d.T, dsplit), 128, 0, st, sbuf, y, row_of, w, d.T, d.k, d.D,
@@ -721,7 +744,8 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     LaunchScope ls_(kKCombineNorm, st);
     const cudaError_t le_ = launch_k(combine_norm_kernel, d.T, kCombThreads, 0, st, sbuf,
                                      reinterpret_cast<const __nv_bfloat16*>(ws + F.y), row_of, w, d.T, d.k, d.D,
-                                     p->rms_norm_out, static_cast<__nv_bfloat16*>(p->out), p->out_f32);
+                                     p->rms_norm_out, nullptr, nullptr, static_cast<__nv_bfloat16*>(p->out),
+                                     p->out_f32);
     MOE_TRY(ls_.done(le_));
   }
   const size_t R = static_cast<size_t>(d.T) * d.k;
@@ -803,6 +827,7 @@ moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out) {
   out->off = L.off;
   out->row_of = L.row_of;
   out->token_of = L.token_of;
+  out->x_norm = L.x_norm;
   return MOE_OK;
 }
 
@@ -1109,7 +1134,7 @@ moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream) {
   MOE_TRY(resolve_workspace(p, s, L, &ws));
   MOE_TRY(enqueue_block(p, d, L, ws, s, st));
   const size_t R = static_cast<size_t>(d.T) * d.k;
-  const void* srcs[3] = {p->x, ws + L.h, ws + L.hs};
+  const void* srcs[3] = {p->norm_pre ? ws + L.x_norm : p->x, ws + L.h, ws + L.hs};
   const size_t ns[3] = {static_cast<size_t>(d.T) * d.D, R * d.F, static_cast<size_t>(d.T) * d.S};
   for (int i = 0; i < 3; ++i) {
     const int blocks = static_cast<int>(std::min<size_t>((ns[i] / 8 + 255) / 256, static_cast<size_t>(s->sm_count) * 8));

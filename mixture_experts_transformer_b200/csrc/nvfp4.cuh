@@ -635,17 +635,19 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
 
 // --------------------------------------------------------------- combine
 
-// out[t] = s[t] + sum_j w[t, j] y[row_of[t, j]] in fp32 (slot order), then
-// optionally x / sqrt(mean(x^2) + 1e-6) (the unlearned RMSNorm between the
-// blocks of the NVFP4 stack; model card: RMSNorm, eps 1e-06). One CTA per
-// token; each thread keeps up to kCombVec 8-column vectors in registers.
+// f[t] = s[t] + sum_j w[t, j] y[row_of[t, j]] in fp32 (slot order), then
+// optionally the RMSNorm f / sqrt(mean(f^2) + 1e-6) (model card: RMSNorm, eps
+// 1e-06) - unlearned between the blocks of the NVFP4 stack, or times a learned
+// scale gamma (the post-FFN norm of the sandwich) - and optionally plus the
+// block's raw input xres (the residual). One CTA per token; each thread keeps
+// up to kCombVec 8-column vectors in registers.
 constexpr int kCombThreads = 128;
 constexpr int kCombVec = 4;  // supports D <= 128 * 4 * 8 = 4096
 
 __global__ void __launch_bounds__(kCombThreads) combine_norm_kernel(
     const float* __restrict__ s, const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ row_of,
-    const float* __restrict__ w, int T, int k, int D, int rms_norm, __nv_bfloat16* __restrict__ out,
-    float* __restrict__ out_f32) {
+    const float* __restrict__ w, int T, int k, int D, int rms_norm, const __nv_bfloat16* __restrict__ gamma,
+    const __nv_bfloat16* __restrict__ xres, __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32) {
   __shared__ int s_row[128];
   __shared__ float s_w[128];
   __shared__ float s_red[kCombThreads / 32];
@@ -694,6 +696,18 @@ __global__ void __launch_bounds__(kCombThreads) combine_norm_kernel(
     float o[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) o[i] = acc[u][i] * scale;
+    if (gamma) {  // learned scale of the normalisation
+      const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
+      const __nv_bfloat16* gb = reinterpret_cast<const __nv_bfloat16*>(&gv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] *= __bfloat162float(gb[i]);
+    }
+    if (xres) {  // residual: the block's raw input
+      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xres + static_cast<size_t>(t) * D) + v);
+      const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(&xv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o[i] = __bfloat162float(xb[i]) + o[i];
+    }
     reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * D)[v] =
         make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
     if (out_f32) {

@@ -53,7 +53,8 @@ def test_workspace_sizes(lib):
     assert big >= 4096 * 8 * (2816 * 2 * 2 + 704 * 2)
     p = B.make_params(64)
     lay = B.moe_workspace_layout(p)
-    offs = [lay.x_perm, lay.h, lay.y, lay.hs, lay.s, lay.idx, lay.w, lay.cnt, lay.off, lay.row_of, lay.token_of]
+    offs = [lay.x_perm, lay.h, lay.y, lay.hs, lay.s, lay.idx, lay.w, lay.cnt, lay.off, lay.row_of, lay.token_of,
+            lay.x_norm]
     assert all(o % 256 == 0 for o in offs)
     assert len(set(offs)) == len(offs)
     assert lay.total_bytes == B.moe_workspace_bytes(64)
@@ -81,6 +82,14 @@ def test_host_validation(lib):
     assert f(p) == B.MOE_ERR_INVALID_ARG
     p = _params()
     p.num_experts = 256  # more than one warp's 4 experts per lane
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params(norm_pre=18)  # misaligned learned scale
+    assert f(p) == B.MOE_ERR_ALIGNMENT
+    p = _params(norm_post=16)
+    p.embed_dim = 4160  # the post-norm keeps a whole row per CTA: embed_dim <= 4096
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params()
+    p.embed_dim, p.residual = 4160, 1
     assert f(p) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_block_forward_ex(None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_timeout_probe(0, None) == B.MOE_ERR_INVALID_ARG
