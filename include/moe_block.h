@@ -100,8 +100,8 @@ typedef enum {
  *   norm_post [embed_dim] bf16: the block output f becomes
  *             norm_post * f / sqrt(mean(f^2) + 1e-6), in fp32;
  *   residual  nonzero: out = RNE(x + that), the raw input x added in fp32.
- * With norm_post or residual, embed_dim must be <= 4096. out_f32 then holds
- * the final pre-rounding value.
+ * With any of the three, embed_dim must be <= 4096 (a row per CTA). out_f32
+ * then holds the final pre-rounding value.
  */
 typedef struct moe_params {
   int T;

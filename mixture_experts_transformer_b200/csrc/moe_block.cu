@@ -374,7 +374,7 @@ moe_status check_block_args(const moe_params* p, Dims* d) {
   const uintptr_t bytes = static_cast<uintptr_t>(d->T) * d->D * 2;
   if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
   if ((p->norm_pre && !aligned16(p->norm_pre)) || (p->norm_post && !aligned16(p->norm_post))) return MOE_ERR_ALIGNMENT;
-  if ((p->norm_post || p->residual) && d->D > kCombThreads * kCombVec * 8) return MOE_ERR_INVALID_ARG;
+  if ((p->norm_pre || p->norm_post || p->residual) && d->D > kCombThreads * kCombVec * 8) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -467,8 +467,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   if (p->norm_pre) {
     __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + L.x_norm);
     LaunchScope ls_(kKPreNorm, st);
-    const int blocks = static_cast<int>(std::min<long long>((d.T + kNormWarps - 1) / kNormWarps, 148LL * 16));
-    MOE_TRY(ls_.done(launch_k(rms_norm_rows_kernel, blocks, kNormWarps * 32, 0, st,
+    MOE_TRY(ls_.done(launch_k(rms_norm_rows_kernel, d.T, kNormThreads, 0, st,
                               static_cast<const __nv_bfloat16*>(p->x),
                               static_cast<const __nv_bfloat16*>(p->norm_pre), d.T, d.D, xn)));
     xin = xn;

@@ -91,5 +91,8 @@ def test_host_validation(lib):
     p = _params()
     p.embed_dim, p.residual = 4160, 1
     assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params(norm_pre=16)
+    p.embed_dim = 4160
+    assert f(p) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_block_forward_ex(None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_timeout_probe(0, None) == B.MOE_ERR_INVALID_ARG
