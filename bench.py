@@ -54,6 +54,14 @@ WORKLOADS = {
         layers=30,
         desc="30 Gemma-4-26B-A4B MoE blocks in NVFP4 (group 16, e4m3 scales), RMSNorm between blocks, T=2048",
     ),
+    "e4b_dense_decode": dict(
+        T=64, bias=False, bound="hbm", dense=True,
+        desc="Gemma-4-E4B dense GeGLU FFN (embed 2560, hidden 10240), T=64 tokens, bf16",
+    ),
+    "e4b_dense": dict(
+        T=4096, bias=False, bound="tensor", dense=True,
+        desc="Gemma-4-E4B dense GeGLU FFN (embed 2560, hidden 10240), T=4096 tokens, bf16",
+    ),
 }
 FP4_TFLOPS_NOMINAL_RATIO = 4.0  # dense fp4 : bf16 tensor throughput, nominal (9 : 2.25 PFLOP/s)
 METRIC = "MoE-block tokens/s"
@@ -709,12 +717,21 @@ def run_reference(args, world, rank):
 
     wl = WORKLOADS[args.workload]
     T = wl["T"]
-    w = inputs.make_weights()
     n = min(T, 8)
-    x = inputs.make_x(n)
-    bias = inputs.zipf_router_bias() if wl["bias"] else None
-    args_w = (w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd)
-    if args.sandwich:
+    metric = METRIC
+    if wl.get("dense"):
+        dw = inputs.make_dense_weights()
+        x = inputs.make_x(n, inputs.E4B_EMBED_DIM)
+        metric = "dense FFN tokens/s"
+        step = lambda: mo.dense_ffn(x, dw.wg, dw.wu, dw.wd)  # noqa: E731
+    else:
+        w = inputs.make_weights()
+        x = inputs.make_x(n)
+        bias = inputs.zipf_router_bias() if wl["bias"] else None
+        args_w = (w.w_router, w.wg, w.wu, w.wd, w.sg, w.su, w.sd)
+    if wl.get("dense"):
+        pass
+    elif args.sandwich:
         from oracle import sandwich as sw
 
         rng = np.random.default_rng(9)
@@ -732,7 +749,7 @@ def run_reference(args, world, rank):
     cores = _oracle_cores()
     return {
         "impl": "reference",
-        "metric": METRIC,
+        "metric": metric,
         "value": v,
         "unit": "tokens/s",
         "n_gpus": world,
@@ -762,6 +779,168 @@ def run_reference(args, world, rank):
     }
 
 
+def run_dense(args, world, rank, local):
+    """One step = the dense GeGLU FFN of the E4B sibling over T tokens."""
+    import torch
+
+    from mixture_experts_transformer_b200 import binding as B
+    from mixture_experts_transformer_b200 import block, build, inputs
+
+    if rank == 0:
+        build.build()
+    barrier(world)
+    B.lib()
+    torch.cuda.set_device(local)
+    wl = WORKLOADS[args.workload]
+    T, Dd, Sd = wl["T"], inputs.E4B_EMBED_DIM, inputs.E4B_HIDDEN_DIM
+    g = torch.Generator(device="cuda").manual_seed(0)
+
+    def rnd(*shape, s=0.02):
+        return torch.empty(shape, device="cuda").normal_(0.0, s, generator=g).to(torch.bfloat16)
+
+    wg, wu, wd = rnd(Dd, Sd), rnd(Dd, Sd), rnd(Sd, Dd)
+    gx = torch.Generator(device="cuda").manual_seed(1 + rank)
+    x = torch.empty((T, Dd), device="cuda").normal_(0.0, 1.0, generator=gx).to(torch.bfloat16)
+    out = torch.empty((T, Dd), dtype=torch.bfloat16, device="cuda")
+    p0 = B.make_dense_params(T, embed_dim=Dd, hidden_dim=Sd)
+    ws = torch.empty(B.moe_dense_workspace_bytes(p0), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    p = B.make_dense_params(T, x, wg, wu, wd, out, embed_dim=Dd, hidden_dim=Sd, workspace=ws)
+    block.dense_forward(x, wg, wu, wd, debug=True, workspace=ws)
+    for _ in range(max(args.warmup, 3)):
+        B.check(B.moe_dense_ffn_forward(p, stream), "dense")
+    torch.cuda.synchronize()
+    launches = B.moe_last_launch_count()
+    # per-kernel breakdown (a separate pass)
+    B.moe_profile_begin()
+    for _ in range(min(args.steps, 50)):
+        B.check(B.moe_dense_ffn_forward(p, stream), "dense")
+    torch.cuda.synchronize()
+    breakdown = B.moe_profile_end()
+    dominant = max(breakdown, key=lambda k: breakdown[k][0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        B.moe_profile_begin([dominant])
+        e0.record(stream)
+        for _ in range(args.steps):
+            B.check(B.moe_dense_ffn_forward(p, stream), "dense")
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per_kernel = B.moe_profile_end()
+    barrier(world)
+    ms = reduce_max(e0.elapsed_time(e1), world)
+    agg = aggregate(T, args.steps, ms, world)
+    if B.moe_get_device_status() != B.MOE_OK:
+        raise RuntimeError("device status after the timed region")
+    # end to end through the public call: pinned host x in, host out back
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((T, Dd), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    pe = B.make_dense_params(T, x_dev, wg, wu, wd, out, embed_dim=Dd, hidden_dim=Sd, workspace=ws)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        B.check(B.moe_dense_ffn_forward(pe, stream), "dense")
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(t0.elapsed_time(t1), world)
+    barrier(world)
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    step_ms = agg["ms_per_step"]
+    flops = 2.0 * 3 * Dd * Sd * T
+    wbytes = 3 * Dd * Sd * 2
+    dom_ms = per_kernel[dominant][0] / per_kernel[dominant][1]
+    if dominant == "grouped_gemm_gateup":
+        dom_bytes, dom_flops = 2 * Dd * Sd * 2 + T * Dd * 2 + T * Sd * 2, 2.0 * 2 * Dd * Sd * T
+    else:
+        dom_bytes, dom_flops = Sd * Dd * 2 + T * Sd * 2 + T * Dd * 2, 2.0 * Dd * Sd * T
+    if wl["bound"] == "hbm":
+        ach, peak, unit, byts = dom_bytes / (dom_ms / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s", dom_bytes
+    else:
+        ach, peak, unit, byts = dom_flops / (dom_ms / 1e3) / 1e12, peaks["bf16_tflops"], "TFLOP/s", dom_bytes
+    res = {
+        "metric": "dense FFN tokens/s",
+        "value": agg["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded N(0,0.02) random-init weights of the published E4B FFN shapes, x ~ N(0,1)",
+        "config": {
+            "workload": wl["desc"],
+            "tokens_per_gpu": T,
+            "global_batch": T * world,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "weights 157 MB, larger than L2",
+        },
+        "roofline": {
+            "bound": wl["bound"],
+            "kernel": dominant,
+            "achieved": ach,
+            "peak": peak,
+            "peak_source": f"{peaks['source']} " + ("hbm_gbs" if wl["bound"] == "hbm" else "bf16_tflops"),
+            "unit": unit,
+            "frac": ach / peak,
+            "traffic": None,
+            "algorithmic_bytes": byts,
+            "kernel_ms": dom_ms,
+        },
+        "block_roofline": {
+            "hbm_weights_gbs": wbytes / (step_ms / 1e3) / 1e9,
+            "hbm_frac": wbytes / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "tensor_tflops": flops / (step_ms / 1e3) / 1e12,
+            "tensor_frac": flops / (step_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        },
+        "kernels_ms_per_launch": {k: v[0] / v[1] for k, v in breakdown.items()},
+        "gpu_launches": launches * args.steps,
+        "e2e": {
+            "value": T * args.steps * world / (e2e_ms / 1e3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": T * Dd * 2,
+            "d2h_bytes_per_step": T * Dd * 2,
+        },
+        "clocks": clocks.report(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import moe_oracle as mo
+
+        wh = [a.float().cpu().numpy() for a in (wg, wu, wd)]
+        xs = x[: min(T, 64)].float().cpu().numpy()
+        done, t0s = 0, time.perf_counter()
+        while True:
+            mo.dense_ffn(xs, *wh)
+            done += xs.shape[0]
+            if time.perf_counter() - t0s > 12.0 or done >= 64 * xs.shape[0]:
+                break
+        el = time.perf_counter() - t0s
+        res["cpu_baseline"] = {
+            "value": done / el,
+            "unit": "tokens/s",
+            "cores": _oracle_cores(),
+            "kind": "oracle",
+            "sample": f"{done} tokens ({done // xs.shape[0]} passes over the first {xs.shape[0]} tokens), {el:.1f} s",
+        }
+    return res
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args.gpus)
@@ -770,6 +949,8 @@ def main():
             res = run_reference(args, world, rank)
         elif args.workload == "nvfp4_stack":
             res = run_stack(args, world, rank, local)
+        elif WORKLOADS[args.workload].get("dense"):
+            res = run_dense(args, world, rank, local)
         else:
             res = run_ours(args, world, rank, local)
         if rank == 0 and res is not None:

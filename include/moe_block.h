@@ -346,6 +346,42 @@ moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream);
  */
 moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream);
 
+/* -------------------------------------------------------- dense GeGLU FFN
+ *
+ * The feed-forward of the dense E4B sibling (gm.nn.Gemma4_E4B
+ * TransformerConfig: embed_dim 2560, hidden_dim 10240, enable_moe=False) - the
+ * same bias-free GeGLU, tanh GELU on the gate projection, as the 26B-A4B
+ * block's shared MLP:
+ *   out = RNE_bf16((gelu_tanh(x Wg) * (x Wu)) Wd), fp32 accumulation, the
+ *   hidden rows stored as bf16 (RNE), as in the block.
+ * Dims left 0 take embed_dim 2560 and hidden_dim 10240; both must be
+ * multiples of 64. Weights bf16, row-major, exactly as given: wg, wu
+ * [embed_dim, hidden_dim], wd [hidden_dim, embed_dim]. x [T, embed_dim] bf16
+ * in, out [T, embed_dim] bf16 out (must not overlap x); out_f32 [T, embed_dim]
+ * fp32 (optional): the pre-rounding output. workspace: at least
+ * moe_dense_workspace_bytes(p) bytes, 256-byte aligned, or NULL for the
+ * library's cached allocation. T = 0 is a no-op; errors as for the block.
+ */
+#define MOE_E4B_EMBED_DIM 2560
+#define MOE_E4B_HIDDEN_DIM 10240
+
+typedef struct moe_dense_params {
+  int T;
+  int embed_dim;
+  int hidden_dim;
+  const void* x;
+  const void* wg;
+  const void* wu;
+  const void* wd;
+  void* out;
+  float* out_f32;
+  void* workspace;
+  size_t workspace_bytes;
+} moe_dense_params;
+
+size_t moe_dense_workspace_bytes(const moe_dense_params* p);
+moe_status moe_dense_ffn_forward(const moe_dense_params* p, void* stream);
+
 /* Human-readable name of a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -369,3 +369,53 @@ def moe_block_forward_nvfp4(p: MoeNvfp4Params, stream=None) -> int:
 
 def moe_nvfp4_calibrate(p: MoeParams, amax, stream=None) -> int:
     return lib().moe_nvfp4_calibrate(ctypes.byref(p), ptr(amax), stream_handle(stream))
+
+
+# ------------------------------------------------------------ dense GeGLU FFN
+
+E4B_EMBED_DIM = 2560
+E4B_HIDDEN_DIM = 10240
+
+
+class MoeDenseParams(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int),
+        ("embed_dim", ctypes.c_int),
+        ("hidden_dim", ctypes.c_int),
+        ("x", _vp),
+        ("wg", _vp),
+        ("wu", _vp),
+        ("wd", _vp),
+        ("out", _vp),
+        ("out_f32", _vp),
+        ("workspace", _vp),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+EXPORTS.update(
+    {
+        "moe_dense_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeDenseParams)]),
+        "moe_dense_ffn_forward": (ctypes.c_int, [ctypes.POINTER(MoeDenseParams), _vp]),
+    }
+)
+
+
+def make_dense_params(T, x=None, wg=None, wu=None, wd=None, out=None, *, embed_dim=0, hidden_dim=0, out_f32=None,
+                      workspace=None) -> MoeDenseParams:
+    p = MoeDenseParams()
+    p.T, p.embed_dim, p.hidden_dim = T, embed_dim, hidden_dim
+    for name, val in (("x", x), ("wg", wg), ("wu", wu), ("wd", wd), ("out", out), ("out_f32", out_f32),
+                      ("workspace", workspace)):
+        setattr(p, name, ptr(val))
+    if workspace is not None:
+        p.workspace_bytes = workspace.numel() * workspace.element_size()
+    return p
+
+
+def moe_dense_workspace_bytes(p: MoeDenseParams) -> int:
+    return lib().moe_dense_workspace_bytes(ctypes.byref(p))
+
+
+def moe_dense_ffn_forward(p: MoeDenseParams, stream=None) -> int:
+    return lib().moe_dense_ffn_forward(ctypes.byref(p), stream_handle(stream))

@@ -214,3 +214,22 @@ def calibrate(dw: DeviceWeights, x: torch.Tensor, top_k: int = B.TOP_K, router_b
     B.check(B.moe_nvfp4_calibrate(p, amax, stream), "moe_nvfp4_calibrate")
     a = amax.cpu().numpy().astype(np.float32)
     return tuple(np.float32(2688.0) / v if v > 0 else np.float32(1.0) for v in a), a
+
+
+# ---------------------------------------------------------------- dense FFN
+
+
+def dense_forward(x: torch.Tensor, wg: torch.Tensor, wu: torch.Tensor, wd: torch.Tensor, *, debug: bool = False,
+                  workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> BlockResult:
+    """The dense GeGLU FFN: out = (gelu_tanh(x wg) * (x wu)) wd; wg, wu [D, S], wd [S, D] bf16."""
+    T, D = x.shape
+    S = wg.shape[1]
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.bfloat16, device=x.device)
+    res = BlockResult(out=out)
+    if debug:
+        res.out_f32 = torch.empty((T, D), dtype=torch.float32, device=x.device)
+    p = B.make_dense_params(T, x, wg, wu, wd, out, embed_dim=D, hidden_dim=S, out_f32=res.out_f32,
+                            workspace=workspace)
+    B.check(B.moe_dense_ffn_forward(p, stream), "moe_dense_ffn_forward")
+    return res

@@ -792,6 +792,110 @@ moe_status noalloc_base(uint8_t** out) {
 
 using namespace moe;
 
+namespace moe {
+namespace {
+
+// ------------------------------------------------------- dense GeGLU FFN
+
+struct DenseDims {
+  int T, D, S;
+};
+
+struct DenseLayout {
+  size_t hs, tiles_gu, tiles_dn, counts, total;
+  int max_gu, max_dn;
+};
+
+DenseDims dense_dims(const moe_dense_params* p) {
+  return DenseDims{p->T, p->embed_dim ? p->embed_dim : MOE_E4B_EMBED_DIM,
+                   p->hidden_dim ? p->hidden_dim : MOE_E4B_HIDDEN_DIM};
+}
+
+bool dense_dims_ok(const DenseDims& d) {
+  return d.T >= 0 && d.D > 0 && d.S > 0 && d.D % 64 == 0 && d.S % 64 == 0 && d.D <= (1 << 20) && d.S <= (1 << 20);
+}
+
+DenseLayout dense_layout(const DenseDims& d) {
+  DenseLayout L{};
+  const size_t mt = (static_cast<size_t>(d.T) + kBM - 1) / kBM;
+  L.max_gu = static_cast<int>(std::max<size_t>(1, mt * ((d.S + 127) / 128)));
+  L.max_dn = static_cast<int>(std::max<size_t>(1, mt * ((d.D + 255) / 256)));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, kAlign);
+    return at;
+  };
+  L.hs = take(static_cast<size_t>(d.T) * d.S * 2);
+  L.tiles_gu = take(static_cast<size_t>(L.max_gu) * sizeof(Tile));
+  L.tiles_dn = take(static_cast<size_t>(L.max_dn) * sizeof(Tile));
+  L.counts = take(sizeof(TileCounts));
+  L.total = o;
+  return L;
+}
+
+moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const DenseLayout& L, uint8_t* ws,
+                         DeviceState* s, cudaStream_t st) {
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(ws + L.hs);
+  TileCounts* counts = reinterpret_cast<TileCounts*>(ws + L.counts);
+  // large batches: paired gate|up (two row blocks per weight stage), down on SM pairs
+  const bool pairs = d.T >= 2 * kBM;
+  const bool pair_dn = pairs && d.D % 128 == 0 && s->pair_clusters_dn > 0;
+  {
+    LaunchScope ls_(kKRouteScan, st);
+    MOE_TRY(ls_.done(launch_k(dense_tiles_kernel, 1, 256, 0, st, d.T, d.S, d.D, pairs ? 1 : 0, pair_dn ? 1 : 0, 256,
+                              reinterpret_cast<Tile*>(ws + L.tiles_gu), reinterpret_cast<Tile*>(ws + L.tiles_dn),
+                              counts)));
+  }
+  GemmParams gu;
+  std::memset(&gu, 0, sizeof(gu));
+  if (!map_2d(&gu.tmA[0], p->x, d.T, d.D, kBM) || !map_3d(&gu.tmB0[0], p->wg, 1, d.D, d.S) ||
+      !map_3d(&gu.tmB1[0], p->wu, 1, d.D, d.S))
+    return MOE_ERR_CUDA;
+  gu.prob[0] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
+  gu.nprob = 1;
+  gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
+  gu.num_tiles = &counts->gateup;
+  gu.next_tile = &counts->next_gateup;
+  gu.err = s->err;
+  {
+    LaunchScope ls_(kKGemmGateUp, st);
+    const int grid = std::min(s->sm_count, L.max_gu);
+    MOE_TRY(ls_.done(pairs ? launch_k(grouped_gemm_kernel<true, true>, grid, kGemmThreads, kGemmSmemBytes, st, gu)
+                           : launch_k(grouped_gemm_kernel<true>, grid, kGemmThreads, kGemmSmemBytes, st, gu)));
+  }
+  GemmParams dn;
+  std::memset(&dn, 0, sizeof(dn));
+  if (!map_2d(&dn.tmA[0], hs, d.T, d.S, kBM) || !map_3d(&dn.tmB0[0], p->wd, 1, d.S, d.D)) return MOE_ERR_CUDA;
+  dn.tmB1[0] = dn.tmB0[0];
+  // with out_f32 the down GEMM writes fp32 and a pass rounds it into out
+  dn.prob[0] = GemmProblem{d.S, d.D, 1, d.T, p->out_f32 ? static_cast<void*>(p->out_f32) : p->out, d.D,
+                           p->out_f32 ? 1 : 0};
+  dn.nprob = 1;
+  dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
+  dn.num_tiles = &counts->down;
+  dn.next_tile = &counts->next_down;
+  dn.err = s->err;
+  {
+    LaunchScope ls_(kKGemmDown, st);
+    const int grid = std::min(s->sm_count, L.max_dn);
+    MOE_TRY(ls_.done(pair_dn ? launch_k(grouped_gemm_pair_kernel<false>, 2 * s->pair_clusters_dn, kGemmThreads,
+                                        kP2SmemBytes, st, dn)
+                             : launch_k(grouped_gemm_kernel<false>, grid, kGemmThreads, kGemmSmemBytes, st, dn)));
+  }
+  if (p->out_f32) {
+    const size_t n8 = static_cast<size_t>(d.T) * d.D / 8;
+    LaunchScope ls_(kKCombine, st);
+    const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, static_cast<size_t>(s->sm_count) * 8));
+    MOE_TRY(ls_.done(launch_k(round_bf16_kernel, blocks, 256, 0, st, static_cast<const float*>(p->out_f32), n8,
+                              static_cast<__nv_bfloat16*>(p->out))));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_bytes_ex(const moe_params* p) {
@@ -1143,6 +1247,45 @@ moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream) {
     MOE_TRY(ls_.done(le_));
   }
   return MOE_OK;
+}
+
+size_t moe_dense_workspace_bytes(const moe_dense_params* p) {
+  if (!p) return 0;
+  const DenseDims d = dense_dims(p);
+  if (!dense_dims_ok(d)) return 0;
+  return dense_layout(d).total;
+}
+
+moe_status moe_dense_ffn_forward(const moe_dense_params* p, void* stream) {
+  t_launches = 0;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  const DenseDims d = dense_dims(p);
+  if (!dense_dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  if (d.T == 0) return MOE_OK;
+  const void* req[] = {p->x, p->wg, p->wu, p->wd, p->out};
+  for (const void* q : req)
+    if (!q) return MOE_ERR_INVALID_ARG;
+  for (const void* q : req)
+    if (!aligned16(q)) return MOE_ERR_ALIGNMENT;
+  if (p->out_f32 && !aligned16(p->out_f32)) return MOE_ERR_ALIGNMENT;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(p->x), ob = reinterpret_cast<uintptr_t>(p->out);
+  const uintptr_t bytes = static_cast<uintptr_t>(d.T) * d.D * 2;
+  if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  const DenseLayout L = dense_layout(d);
+  uint8_t* ws = nullptr;
+  if (p->workspace) {
+    if ((reinterpret_cast<uintptr_t>(p->workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGNMENT;
+    if (p->workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    ws = static_cast<uint8_t*>(p->workspace);
+  } else {
+    void* w = nullptr;
+    MOE_TRY(library_workspace(s, L.total, &w));
+    ws = static_cast<uint8_t*>(w);
+  }
+  return enqueue_dense(p, d, L, ws, s, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

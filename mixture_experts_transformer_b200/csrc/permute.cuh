@@ -185,6 +185,49 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   }
 }
 
+// Work tiles of a dense feed-forward (one problem, no routing): rows [0, T)
+// in 128-row blocks (pairs of blocks when pair), column tiles 128 wide per
+// projection for gate|up and dn_cols wide for down. Also clears the GEMMs'
+// work counters. One CTA.
+__global__ void __launch_bounds__(256) dense_tiles_kernel(int T, int S, int D, int pair_gu, int pair_dn,
+                                                          int dn_cols, Tile* __restrict__ tiles_gu,
+                                                          Tile* __restrict__ tiles_dn,
+                                                          TileCounts* __restrict__ counts) {
+  pdl_wait_then_release();
+  const int mt = (T + kBM - 1) / kBM;
+  auto emit = [&](Tile* tiles, int pair, int ncol, int cw) -> int {
+    const int mstep = pair ? 2 : 1;
+    const int pt = (mt + mstep - 1) / mstep;
+    for (int i = threadIdx.x; i < ncol * pt; i += blockDim.x) {
+      const int nt = i / pt, m = (i % pt) * mstep;
+      const int r1 = pair ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
+      tiles[i] = Tile{0, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, {0, 0}};
+    }
+    return ncol * pt;
+  };
+  const int n_gu = emit(tiles_gu, pair_gu, (S + 127) / 128, 128);
+  const int n_dn = emit(tiles_dn, pair_dn, (D + dn_cols - 1) / dn_cols, dn_cols);
+  if (threadIdx.x == 0) {
+    counts->gateup = n_gu;
+    counts->down = n_dn;
+    counts->next_gateup = 0;
+    counts->next_down = 0;
+  }
+}
+
+// fp32 -> bf16 (round to nearest even), 8 values per thread.
+__global__ void __launch_bounds__(256) round_bf16_kernel(const float* __restrict__ src, size_t n8,
+                                                         __nv_bfloat16* __restrict__ dst) {
+  pdl_wait_then_release();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
+    const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+    reinterpret_cast<uint4*>(dst)[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                  pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
 // One warp per (token, slot): its routed row from the bitmasks; lane 0 writes
 // row_of / token_of, and (when x is given) the warp copies x[t] into
 // x_perm[row] with 16-byte vectors, so the GEMM's A tiles are plain boxes.

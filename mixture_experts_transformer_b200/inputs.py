@@ -101,6 +101,30 @@ def make_weights(dims: Dims = GEMMA4_26B_A4B, seed: int = 0, std: float = INIT_S
     )
 
 
+# The dense E4B sibling (gm.nn.Gemma4_E4B TransformerConfig: embed_dim 2560,
+# hidden_dim 10240, enable_moe=False).
+E4B_EMBED_DIM = 2560
+E4B_HIDDEN_DIM = 10240
+
+
+@dataclasses.dataclass
+class DenseWeights:
+    wg: np.ndarray  # [D, S]
+    wu: np.ndarray  # [D, S]
+    wd: np.ndarray  # [S, D]
+
+
+def make_dense_weights(embed_dim: int = E4B_EMBED_DIM, hidden_dim: int = E4B_HIDDEN_DIM, seed: int = 0,
+                       std: float = INIT_STD) -> DenseWeights:
+    """Gate, up, down of a dense GeGLU FFN from one seeded stream, N(0, std^2) -> bf16 bits."""
+    rng = _generator(seed)
+    return DenseWeights(
+        wg=_normal_bf16(rng, (embed_dim, hidden_dim), std),
+        wu=_normal_bf16(rng, (embed_dim, hidden_dim), std),
+        wd=_normal_bf16(rng, (hidden_dim, embed_dim), std),
+    )
+
+
 def make_x(tokens: int, embed_dim: int = EMBED_DIM, seed: int = 1) -> np.ndarray:
     return _normal_bf16(_generator(seed), (tokens, embed_dim), 1.0)
 

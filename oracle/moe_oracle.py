@@ -157,6 +157,14 @@ def geglu_ffn(x, w_gate, w_up, w_down) -> np.ndarray:
 # ------------------------------------------------------------------- block
 
 
+def dense_ffn(x, w_gate, w_up, w_down) -> np.ndarray:
+    """The feed-forward of the dense E4B sibling [gm.nn.Gemma4_E4B TransformerConfig:
+    enable_moe=False, hidden_dim=10240, embed_dim=2560]: the same bias-free
+    GeGLU as the 26B-A4B block's shared MLP (reading: the pages give the E4B
+    config only; its FFN is the family's gated FFN with gelu_pytorch_tanh)."""
+    return geglu_ffn(x, w_gate, w_up, w_down)
+
+
 def moe_block(x, w_router, wg, wu, wd, sg, su, sd, top_k: int = 8, bias=None, routing=None):
     """out = shared_mlp(x) + sum_k w[t, k] * expert_{idx[t, k]}(x[t]).
 
