@@ -442,7 +442,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
   LaunchScope ls_(kKRouteScatter, st);
   const cudaError_t le_ = launch_k(route_scatter_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E, d.D,
                                    static_cast<const __nv_bfloat16*>(x), row_of, token_of,
-                                   reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm));
+                                   reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm), R, s->err);
   return ls_.done(le_);
 }
 
@@ -527,14 +527,15 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
     // the post-FFN norm and / or the residual need a token's whole row: one CTA per token
     LaunchScope ls_(kKCombineNorm, st);
     MOE_TRY(ls_.done(launch_k(combine_norm_kernel, d.T, kCombThreads, 0, st, sbuf, y, row_of, w, d.T, d.k, d.D,
-                              p->norm_post ? 1 : 0, static_cast<const __nv_bfloat16*>(p->norm_post),
+                              static_cast<int>(R), p->norm_post ? 1 : 0,
+                              static_cast<const __nv_bfloat16*>(p->norm_post),
                               p->residual ? static_cast<const __nv_bfloat16*>(p->x) : nullptr,
-                              static_cast<__nv_bfloat16*>(p->out), p->out_f32)));
+                              static_cast<__nv_bfloat16*>(p->out), p->out_f32, s->err)));
   } else {
   LaunchScope ls_(kKCombine, st);
   const int dsplit = std::max(1, std::min(4, (2 * s->sm_count) / std::max(1, d.T)));
   const cudaError_t le_ = launch_k(combine_kernel, dim3(d.T, dsplit), 128, 0, st, sbuf, y, row_of, w, d.T, d.k, d.D,
-                                                    static_cast<__nv_bfloat16*>(p->out), p->out_f32);
+                                   static_cast<int>(R), static_cast<__nv_bfloat16*>(p->out), p->out_f32, s->err);
   MOE_TRY(ls_.done(le_));
   }
 
@@ -690,7 +691,8 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     LaunchScope ls_(kKScatterFp4, st);
     const cudaError_t le_ = launch_k(route_scatter_fp4_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E,
                                      d.D, static_cast<const __nv_bfloat16*>(p->x), p->g_x, row_of,
-                                     ws + F.xq_perm, ws + F.xsf_perm, ws + F.xq_tok, ws + F.xsf_tok);
+                                     ws + F.xq_perm, ws + F.xsf_perm, ws + F.xq_tok, ws + F.xsf_tok,
+                                     static_cast<int>(F.r_pad), s->err);
     MOE_TRY(ls_.done(le_));
   }
   const long long rp = F.r_pad, tp = F.t_pad;
@@ -743,8 +745,8 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     LaunchScope ls_(kKCombineNorm, st);
     const cudaError_t le_ = launch_k(combine_norm_kernel, d.T, kCombThreads, 0, st, sbuf,
                                      reinterpret_cast<const __nv_bfloat16*>(ws + F.y), row_of, w, d.T, d.k, d.D,
-                                     p->rms_norm_out, nullptr, nullptr, static_cast<__nv_bfloat16*>(p->out),
-                                     p->out_f32);
+                                     static_cast<int>(F.r_pad), p->rms_norm_out, nullptr, nullptr,
+                                     static_cast<__nv_bfloat16*>(p->out), p->out_f32, s->err);
     MOE_TRY(ls_.done(le_));
   }
   const size_t R = static_cast<size_t>(d.T) * d.k;

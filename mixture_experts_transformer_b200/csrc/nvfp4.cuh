@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(256) route_scatter_fp4_kernel(
     const int32_t* __restrict__ idx, const uint32_t* __restrict__ masks, const int32_t* __restrict__ base, int T,
     int k, int E, int D, const __nv_bfloat16* __restrict__ x, float g_x, int32_t* __restrict__ row_of,
     uint8_t* __restrict__ xq_perm, uint8_t* __restrict__ xsf_perm, uint8_t* __restrict__ xq_tok,
-    uint8_t* __restrict__ xsf_tok) {
+    uint8_t* __restrict__ xsf_tok, int rows, uint32_t* __restrict__ err) {
   __shared__ int s_rows[8][128];  // k <= num_experts <= 128
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -200,7 +200,12 @@ __global__ void __launch_bounds__(256) route_scatter_fp4_kernel(
         const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
         const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
         row = __ldg(base + cw) + __popc(below);
-        row_of[a] = row;
+        if (row < 0 || row >= rows) {  // never write outside the routed-row buffers
+          atomicOr(err, kErrBadIndex);
+          row = -1;
+        } else {
+          row_of[a] = row;
+        }
       }
       s_rows[wid][j] = row;
     }
@@ -646,16 +651,24 @@ constexpr int kCombVec = 4;  // supports D <= 128 * 4 * 8 = 4096
 
 __global__ void __launch_bounds__(kCombThreads) combine_norm_kernel(
     const float* __restrict__ s, const __nv_bfloat16* __restrict__ y, const int32_t* __restrict__ row_of,
-    const float* __restrict__ w, int T, int k, int D, int rms_norm, const __nv_bfloat16* __restrict__ gamma,
-    const __nv_bfloat16* __restrict__ xres, __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32) {
+    const float* __restrict__ w, int T, int k, int D, int rows, int rms_norm, const __nv_bfloat16* __restrict__ gamma,
+    const __nv_bfloat16* __restrict__ xres, __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32,
+    uint32_t* __restrict__ err) {
   __shared__ int s_row[128];
   __shared__ float s_w[128];
   __shared__ float s_red[kCombThreads / 32];
   pdl_wait_then_release();
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < k; j += blockDim.x) {
-    s_row[j] = row_of[static_cast<size_t>(t) * k + j];
-    s_w[j] = w[static_cast<size_t>(t) * k + j];
+    int r = row_of[static_cast<size_t>(t) * k + j];
+    float wj = w[static_cast<size_t>(t) * k + j];
+    if (r < 0 || r >= rows) {  // a routed row outside y: report, never address it
+      atomicOr(err, kErrBadIndex);
+      r = 0;
+      wj = 0.f;
+    }
+    s_row[j] = r;
+    s_w[j] = wj;
   }
   __syncthreads();
   const int nvec = D >> 3;

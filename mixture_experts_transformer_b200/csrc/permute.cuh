@@ -237,7 +237,8 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
                                                             int D, const __nv_bfloat16* __restrict__ x,
                                                             int32_t* __restrict__ row_of,
                                                             int32_t* __restrict__ token_of,
-                                                            __nv_bfloat16* __restrict__ x_perm) {
+                                                            __nv_bfloat16* __restrict__ x_perm, long long rows,
+                                                            uint32_t* __restrict__ err) {
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const long long R = static_cast<long long>(T) * k;
@@ -249,6 +250,10 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
     const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
     const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
     const int row = __ldg(base + cw) + __popc(below);
+    if (row < 0 || row >= rows) {  // never write outside the routed-row buffers
+      if (lane == 0) atomicOr(err, kErrBadIndex);
+      continue;
+    }
     if (lane == 0) {
       row_of[a] = row;
       token_of[row] = t;
@@ -266,15 +271,23 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
 // dsplit): CTA (t, q) handles the q-th slice of the row's 8-column vectors.
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ s, const __nv_bfloat16* __restrict__ y,
                                                      const int32_t* __restrict__ row_of,
-                                                     const float* __restrict__ w, int T, int k, int D,
-                                                     __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32) {
+                                                     const float* __restrict__ w, int T, int k, int D, int rows,
+                                                     __nv_bfloat16* __restrict__ out, float* __restrict__ out_f32,
+                                                     uint32_t* __restrict__ err) {
   __shared__ int s_row[128];
   __shared__ float s_w[128];
   pdl_wait_then_release();
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < k; j += blockDim.x) {
-    s_row[j] = row_of[static_cast<size_t>(t) * k + j];
-    s_w[j] = w[static_cast<size_t>(t) * k + j];
+    int r = row_of[static_cast<size_t>(t) * k + j];
+    float wj = w[static_cast<size_t>(t) * k + j];
+    if (r < 0 || r >= rows) {  // a routed row outside y: report, never address it
+      atomicOr(err, kErrBadIndex);
+      r = 0;
+      wj = 0.f;
+    }
+    s_row[j] = r;
+    s_w[j] = wj;
   }
   __syncthreads();
   const int nvec = D >> 3;

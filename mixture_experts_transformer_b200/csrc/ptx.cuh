@@ -15,7 +15,7 @@ namespace moe {
 enum : uint32_t {
   kErrWaitTimeout = 1u,  // a bounded mbarrier / flag wait ran out
   kErrBadTile = 2u,      // a work-list entry failed its range check
-  kErrBadIndex = 4u,     // an expert index outside [0, num_experts)
+  kErrBadIndex = 4u,     // an expert index outside [0, num_experts), or a routed row outside its buffer
 };
 
 // Nanoseconds a kernel waits on one barrier phase before it gives up.
