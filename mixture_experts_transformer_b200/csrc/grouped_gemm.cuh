@@ -60,9 +60,10 @@ struct __align__(16) Tile {
   int32_t row0;   // first A row
   int32_t rows;   // rows of A that belong to this tile (1..128)
   int32_t n0;     // first output column (per projection for GATEUP)
-  int32_t row1;   // PAIRED: first row of the second 128-row block
+  int32_t row1;   // PAIRED: first row of the second 128-row block; split-K tiles: the split
   int32_t rows1;  // PAIRED: its rows (0: no second block)
-  int32_t pad[2];
+  int32_t kb0;    // first 64-deep K block
+  int32_t kbn;    // K blocks of the tile (0: the whole reduction)
 };
 
 struct GemmProblem {
@@ -73,6 +74,9 @@ struct GemmProblem {
   void* out;    // [a_rows, ldo] bf16 or fp32
   int ldo;
   int out_f32;
+  // split-K (down GEMM, fp32 out): a tile with kbn != 0 adds up K blocks
+  // [kb0, kb0 + kbn) only and writes its partial sums at out + row1 * split_stride
+  long long split_stride;
 };
 
 struct GemmParams {
@@ -189,8 +193,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const bool bad_p = p >= P.nprob;
       const GemmProblem& pr = P.prob[bad_p ? 0 : p];
       const bool has1 = PAIRED && tile.rows1 > 0;
+      const int kb_all = pr.K / kBK;
       if (bad_p || g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || tile.rows < 1 || tile.rows > kBM ||
-          tile.n0 < 0 || tile.n0 >= pr.N || (has1 && (tile.row1 < 0 || tile.row1 >= pr.a_rows || tile.rows1 > kBM))) {
+          tile.n0 < 0 || tile.n0 >= pr.N || (has1 && (tile.row1 < 0 || tile.row1 >= pr.a_rows || tile.rows1 > kBM)) ||
+          tile.kb0 < 0 || tile.kbn < 0 || tile.kb0 + (tile.kbn ? tile.kbn : kb_all) > kb_all ||
+          (tile.kbn && (GATEUP || !pr.out_f32 || tile.row1 < 0))) {
         if (lane == 0) {
           atomicOr(P.err, kErrBadTile);
           *abort_flag = 1;
@@ -201,9 +208,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const int cpp = wn >> 6;  // 64-column chunks per projection
       const int nch = GATEUP ? 2 * cpp : cpp;
       const uint32_t bytes = (has1 ? 2 : 1) * kAStageBytes + nch * kBChunkBytes;
-      const int nkb = pr.K / kBK;
+      const int kb_end = tile.kbn ? tile.kb0 + tile.kbn : kb_all;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = tile.kb0; kb < kb_end; ++kb) {
         int waited = 1;
         if (lane == 0) {
           waited = mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err);
@@ -271,14 +278,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         const int wn = tile_cols<GATEUP>(pr, tile.n0);
         const int n_mma = GATEUP ? 2 * wn : wn;
         const uint32_t idesc = idesc_bf16_m128(n_mma, 1);
-        const int nkb = pr.K / kBK;
+        const int kb_end = tile.kbn ? tile.kb0 + tile.kbn : pr.K / kBK;
         const bool has1 = PAIRED && tile.rows1 > 0;
         if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag, P.err)) break;
         if (PAIRED && !mbar_wait(&acc_empty[1], acc_ph ^ 1, abort_flag, P.err)) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = tile.kb0; kb < kb_end; ++kb) {
+          const uint32_t acc_in = kb != tile.kb0;  // the tile's first K block overwrites the accumulator
           if (!mbar_wait(&full[s], ph, abort_flag, P.err)) {
             ok = false;
             break;
@@ -293,9 +301,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
             // B: N-major; 8 K-rows form a 1024 B swizzle atom (SBO), 64-column
             // chunks are 8 KB apart (LBO); +16 K-rows = +2048 B.
             const uint64_t bd = sdesc_sw128(b_addr + k * 2048, kBChunkBytes, 1024);
-            umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            umma_f16(d_tmem, ad, bd, idesc, acc_in | (k != 0));
             if (has1) umma_f16(tmem_base + kAccCols, sdesc_sw128(a_addr + kAStageBytes + k * 32, 16, 1024), bd, idesc,
-                               (kb | k) != 0);
+                               acc_in | (k != 0));
           }
           any = true;
           umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
@@ -380,8 +388,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           tmem_ld_32x32b_x32(tbase + j, a);
           tmem_ld_wait();
           if (pr.out_f32) {
-            store_rows_f32x32(stg, a, lane, reinterpret_cast<float*>(pr.out) + wrow * pr.ldo + tile.n0 + j, pr.ldo,
-                              rows_valid);
+            float* of = reinterpret_cast<float*>(pr.out) + (tile.kbn ? tile.row1 * pr.split_stride : 0);
+            store_rows_f32x32(stg, a, lane, of + wrow * pr.ldo + tile.n0 + j, pr.ldo, rows_valid);
           } else {
             uint32_t pk[16];
 #pragma unroll

@@ -804,8 +804,9 @@ struct DenseDims {
 };
 
 struct DenseLayout {
-  size_t hs, tiles_gu, tiles_dn, counts, total;
+  size_t hs, tiles_gu, tiles_dn, counts, part, total;
   int max_gu, max_dn;
+  int dn_ksplit;  // K splits of the down GEMM (1: none)
 };
 
 DenseDims dense_dims(const moe_dense_params* p) {
@@ -817,11 +818,25 @@ bool dense_dims_ok(const DenseDims& d) {
   return d.T >= 0 && d.D > 0 && d.S > 0 && d.D % 64 == 0 && d.S % 64 == 0 && d.D <= (1 << 20) && d.S <= (1 << 20);
 }
 
+// Small batches leave most SMs without a down tile (one 128-row block gives
+// embed_dim / 256 tiles, 10 at embed_dim 2560, each streaming hidden_dim x 256
+// weights): cut the reduction so that about one wave of (tile, K range) work
+// items covers the device, at least 4 K blocks each. Large batches (paired
+// GEMMs) never split.
+int dense_down_ksplit(const DenseDims& d) {
+  if (d.T >= 2 * kBM) return 1;
+  const long long tiles = ((d.T + kBM - 1) / kBM) * static_cast<long long>((d.D + 255) / 256);
+  const long long by_sm = kSmCountHint / std::max(1LL, tiles);
+  const long long by_k = (d.S / 64) / 4;
+  return static_cast<int>(std::max(1LL, std::min(by_sm, by_k)));
+}
+
 DenseLayout dense_layout(const DenseDims& d) {
   DenseLayout L{};
   const size_t mt = (static_cast<size_t>(d.T) + kBM - 1) / kBM;
+  L.dn_ksplit = dense_down_ksplit(d);
   L.max_gu = static_cast<int>(std::max<size_t>(1, mt * ((d.S + 127) / 128)));
-  L.max_dn = static_cast<int>(std::max<size_t>(1, mt * ((d.D + 255) / 256)));
+  L.max_dn = static_cast<int>(std::max<size_t>(1, mt * ((d.D + 255) / 256) * L.dn_ksplit));
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -832,6 +847,7 @@ DenseLayout dense_layout(const DenseDims& d) {
   L.tiles_gu = take(static_cast<size_t>(L.max_gu) * sizeof(Tile));
   L.tiles_dn = take(static_cast<size_t>(L.max_dn) * sizeof(Tile));
   L.counts = take(sizeof(TileCounts));
+  L.part = take(L.dn_ksplit > 1 ? static_cast<size_t>(L.dn_ksplit) * d.T * d.D * 4 : 0);
   L.total = o;
   return L;
 }
@@ -846,8 +862,8 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   {
     LaunchScope ls_(kKRouteScan, st);
     MOE_TRY(ls_.done(launch_k(dense_tiles_kernel, 1, 256, 0, st, d.T, d.S, d.D, pairs ? 1 : 0, pair_dn ? 1 : 0, 256,
-                              reinterpret_cast<Tile*>(ws + L.tiles_gu), reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                              counts)));
+                              L.dn_ksplit, reinterpret_cast<Tile*>(ws + L.tiles_gu),
+                              reinterpret_cast<Tile*>(ws + L.tiles_dn), counts)));
   }
   GemmParams gu;
   std::memset(&gu, 0, sizeof(gu));
@@ -870,9 +886,15 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   std::memset(&dn, 0, sizeof(dn));
   if (!map_2d(&dn.tmA[0], hs, d.T, d.S, kBM) || !map_3d(&dn.tmB0[0], p->wd, 1, d.S, d.D)) return MOE_ERR_CUDA;
   dn.tmB1[0] = dn.tmB0[0];
-  // with out_f32 the down GEMM writes fp32 and a pass rounds it into out
-  dn.prob[0] = GemmProblem{d.S, d.D, 1, d.T, p->out_f32 ? static_cast<void*>(p->out_f32) : p->out, d.D,
-                           p->out_f32 ? 1 : 0};
+  // split K: the down GEMM writes fp32 partial sums per K range and a pass adds
+  // them up in order and rounds; otherwise, with out_f32, it writes fp32 and a
+  // pass rounds it into out; else it writes the bf16 out itself
+  const bool split = L.dn_ksplit > 1;
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  dn.prob[0] = GemmProblem{d.S, d.D, 1, d.T,
+                           split ? static_cast<void*>(part)
+                                 : (p->out_f32 ? static_cast<void*>(p->out_f32) : p->out),
+                           d.D, (split || p->out_f32) ? 1 : 0, static_cast<long long>(d.T) * d.D};
   dn.nprob = 1;
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
@@ -885,7 +907,13 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
                                         kP2SmemBytes, st, dn)
                              : launch_k(grouped_gemm_kernel<false>, grid, kGemmThreads, kGemmSmemBytes, st, dn)));
   }
-  if (p->out_f32) {
+  if (split) {
+    const size_t n4 = static_cast<size_t>(d.T) * d.D / 4;
+    LaunchScope ls_(kKCombine, st);
+    const int blocks = static_cast<int>(std::min<size_t>((n4 + 255) / 256, static_cast<size_t>(s->sm_count) * 8));
+    MOE_TRY(ls_.done(launch_k(reduce_splits_kernel, blocks, 256, 0, st, static_cast<const float*>(part), L.dn_ksplit,
+                              n4, p->out_f32, static_cast<__nv_bfloat16*>(p->out))));
+  } else if (p->out_f32) {
     const size_t n8 = static_cast<size_t>(d.T) * d.D / 8;
     LaunchScope ls_(kKCombine, st);
     const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, static_cast<size_t>(s->sm_count) * 8));

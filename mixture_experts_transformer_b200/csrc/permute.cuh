@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     for (int i = threadIdx.x; i < n_sh; i += kScanThreads) {
       const int nt = i / pt_sh, m = (i % pt_sh) * mstep;
       const int r1 = pair ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
-      tiles[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, {0, 0}};
+      tiles[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, 0, 0};
     }
     // expert tiles, spread over all threads (one expert may own most of them):
     // flat index f -> expert by binary search over the tile-offset prefix
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
       const int nt = i / pt, m = (i % pt) * mstep;
       const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
       const int r1 = pair ? max(0, min(kBM, ce - (m + 1) * kBM)) : 0;
-      tiles[n_sh + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * cw, rb + (m + 1) * kBM, r1, {0, 0}};
+      tiles[n_sh + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * cw, rb + (m + 1) * kBM, r1, 0, 0};
     }
     return n_sh + n_e;
   };
@@ -187,10 +187,13 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
 
 // Work tiles of a dense feed-forward (one problem, no routing): rows [0, T)
 // in 128-row blocks (pairs of blocks when pair), column tiles 128 wide per
-// projection for gate|up and dn_cols wide for down. Also clears the GEMMs'
-// work counters. One CTA.
+// projection for gate|up and dn_cols wide for down. With dn_ksplit > 1 (small
+// batches, too few down tiles to occupy the GPU) every down tile is cut along
+// the reduction into dn_ksplit K ranges of S / 64 / dn_ksplit blocks (+-1),
+// each writing its own fp32 partial sums. Also clears the GEMMs' work
+// counters. One CTA.
 __global__ void __launch_bounds__(256) dense_tiles_kernel(int T, int S, int D, int pair_gu, int pair_dn,
-                                                          int dn_cols, Tile* __restrict__ tiles_gu,
+                                                          int dn_cols, int dn_ksplit, Tile* __restrict__ tiles_gu,
                                                           Tile* __restrict__ tiles_dn,
                                                           TileCounts* __restrict__ counts) {
   pdl_wait_then_release();
@@ -201,17 +204,53 @@ __global__ void __launch_bounds__(256) dense_tiles_kernel(int T, int S, int D, i
     for (int i = threadIdx.x; i < ncol * pt; i += blockDim.x) {
       const int nt = i / pt, m = (i % pt) * mstep;
       const int r1 = pair ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
-      tiles[i] = Tile{0, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, {0, 0}};
+      tiles[i] = Tile{0, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, 0, 0};
     }
     return ncol * pt;
   };
   const int n_gu = emit(tiles_gu, pair_gu, (S + 127) / 128, 128);
-  const int n_dn = emit(tiles_dn, pair_dn, (D + dn_cols - 1) / dn_cols, dn_cols);
+  int n_dn;
+  if (dn_ksplit > 1) {
+    // (column tile, split) pairs, row blocks innermost: the blocks of a split share its weights
+    const int ncol = (D + dn_cols - 1) / dn_cols, nkb = S / 64;
+    n_dn = ncol * dn_ksplit * mt;
+    for (int i = threadIdx.x; i < n_dn; i += blockDim.x) {
+      const int m = i % mt, q = i / mt, sp = q % dn_ksplit, nt = q / dn_ksplit;
+      const int k0 = static_cast<int>(static_cast<long long>(sp) * nkb / dn_ksplit);
+      const int k1 = static_cast<int>(static_cast<long long>(sp + 1) * nkb / dn_ksplit);
+      tiles_dn[i] = Tile{0, m * kBM, min(kBM, T - m * kBM), nt * dn_cols, sp, 0, k0, k1 - k0};
+    }
+  } else {
+    n_dn = emit(tiles_dn, pair_dn, (D + dn_cols - 1) / dn_cols, dn_cols);
+  }
   if (threadIdx.x == 0) {
     counts->gateup = n_gu;
     counts->down = n_dn;
     counts->next_gateup = 0;
     counts->next_down = 0;
+  }
+}
+
+// dst = RNE_bf16(part[0] + part[1] + ... + part[nsplit-1]), summed in split
+// order in fp32 (deterministic); out_f32 (optional) gets the fp32 sums. Four
+// values per thread.
+__global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restrict__ part, int nsplit, size_t n4,
+                                                            float* __restrict__ out_f32,
+                                                            __nv_bfloat16* __restrict__ dst) {
+  pdl_wait_then_release();
+  const size_t stride4 = n4;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float4 a = reinterpret_cast<const float4*>(part)[i];
+    for (int sp = 1; sp < nsplit; ++sp) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(part) + sp * stride4 + i);
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    if (out_f32) reinterpret_cast<float4*>(out_f32)[i] = a;
+    reinterpret_cast<uint2*>(dst)[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
   }
 }
 

@@ -59,6 +59,13 @@ def test_dense_small_dims(T):
     _check(256, 320, T, std=0.05)
 
 
+@pytest.mark.parametrize("T", [1, 20, 200])
+def test_dense_split_k(T):
+    """hidden 2048 at small batches: the down GEMM is cut along its reduction
+    (8 K ranges of 4 blocks) and the fp32 partial sums are added in order."""
+    _check(256, 2048, T, std=0.05)
+
+
 def test_dense_e4b_decode():
     _check(inputs.E4B_EMBED_DIM, inputs.E4B_HIDDEN_DIM, 64, std=inputs.INIT_STD)
 
