@@ -85,6 +85,9 @@ struct GemmParams {
   CUtensorMap tmB1[2];  // [groups, K, N] bf16 (up; GATEUP only)
   GemmProblem prob[2];
   int nprob;
+  // 1: every weight tile is read by one row block (small batches), so B loads
+  // carry an L2 evict-first policy and the activations keep the cache
+  int stream_weights;
   const Tile* tiles;
   const int32_t* num_tiles;
   int32_t* next_tile;  // work counter, zero at launch: CTAs take tiles in list order as they free up
@@ -169,6 +172,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     int rs = 0;
     uint32_t rph = 0;
     int ti = 0;
+    const uint64_t wpol = l2_policy_evict_first();  // streamed weights go before activations
     if (lane == 0) ti = atomicAdd(P.next_tile, 1);
     ti = __shfl_sync(0xffffffffu, ti, 0);
     while (true) {
@@ -226,8 +230,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           for (int c = 0; c < nch; ++c) {
             const bool up = GATEUP && c >= cpp;
             const int col = tile.n0 + (up ? c - cpp : c) * 64;
-            tma_load_3d(sB + s * kBStageBytes + c * kBChunkBytes, up ? &P.tmB1[p] : &P.tmB0[p], &full[s], col,
-                        kb * kBK, g);
+            void* dst = sB + s * kBStageBytes + c * kBChunkBytes;
+            const CUtensorMap* mb = up ? &P.tmB1[p] : &P.tmB0[p];
+            if (P.stream_weights)
+              tma_load_3d_hint(dst, mb, &full[s], col, kb * kBK, g, wpol);
+            else
+              tma_load_3d(dst, mb, &full[s], col, kb * kBK, g);
           }
         }
         ++issued;

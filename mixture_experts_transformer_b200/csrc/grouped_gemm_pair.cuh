@@ -96,6 +96,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // ------------------------------------------------------ TMA producer
       int s = 0, issued = 0;
       uint32_t ph = 0;
+      const uint64_t wpol = l2_policy_evict_first();  // streamed weights go before activations
       for (int ti = cid; ti < num_tiles; ti += ncl) {
         const Tile tile = P.tiles[ti];
         const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
@@ -127,7 +128,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t bar = full_even + 8u * s;
           if (my_a) tma_load_2d_pair(sA + s * kP2AStage, &P.tmA[p], bar, kb * kBK, row);
           for (int c = 0; c < nch; ++c)
-            tma_load_3d_pair(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g);
+            if (P.stream_weights)
+              tma_load_3d_pair_hint(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g, wpol);
+            else
+              tma_load_3d_pair(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g);
           ++issued;
           if (++s == kP2Stages) {
             s = 0;

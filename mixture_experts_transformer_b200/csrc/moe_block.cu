@@ -44,6 +44,13 @@ struct Layout {
   int nsplit, nchunks, max_tiles_gu, max_tiles_dn;
 };
 
+// Small batches (experts average at most half a 128-row block) read every
+// expert weight tile from one row block: the GEMMs then stream the weights
+// with an L2 evict-first policy. (Measured: decode T=64 0.288 -> 0.281 ms; at
+// T=4096, where an expert's row blocks share its weight tiles through L2, the
+// same policy cost 0.707 -> 0.725 ms.)
+bool stream_weights(const Dims& d) { return static_cast<long long>(d.T) * d.k * 2 <= static_cast<long long>(kBM) * d.E; }
+
 // Large batches (experts average >= 160 routed rows) use the paired gate|up GEMM.
 bool paired_gateup(const Dims& d) { return static_cast<long long>(d.T) * d.k >= 160LL * d.E; }
 // The paired down GEMM pays off later (measured: at ~256 rows per expert it is
@@ -485,6 +492,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   gu.prob[0] = GemmProblem{d.D, d.F, d.E, static_cast<int>(R), h, d.F, 0};
   gu.prob[1] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
   gu.nprob = 2;
+  gu.stream_weights = stream_weights(d) ? 1 : 0;
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
   gu.next_tile = &counts->next_gateup;
@@ -509,6 +517,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   dn.prob[0] = GemmProblem{d.F, d.D, d.E, static_cast<int>(R), y, d.D, 0};
   dn.prob[1] = GemmProblem{d.S, d.D, 1, d.T, sbuf, d.D, 1};
   dn.nprob = 2;
+  dn.stream_weights = gu.stream_weights;
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
   dn.next_tile = &counts->next_down;
@@ -872,6 +881,7 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
     return MOE_ERR_CUDA;
   gu.prob[0] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
   gu.nprob = 1;
+  gu.stream_weights = d.T <= kBM ? 1 : 0;  // one row block reads each weight tile once
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
   gu.next_tile = &counts->next_gateup;
@@ -896,6 +906,7 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
                                  : (p->out_f32 ? static_cast<void*>(p->out_f32) : p->out),
                            d.D, (split || p->out_f32) ? 1 : 0, static_cast<long long>(d.T) * d.D};
   dn.nprob = 1;
+  dn.stream_weights = gu.stream_weights;
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
   dn.next_tile = &counts->next_down;
