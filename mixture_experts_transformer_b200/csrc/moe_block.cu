@@ -422,8 +422,12 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
     MOE_TRY(ls_.done(le_));
   }
   LaunchScope ls_(kKRouterTopk, st);
-  const cudaError_t le_ = launch_k(router_topk_kernel, (d.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
-                                                                                     L.nsplit, d.k, idx, w, masks);
+  const int tk_blocks = (d.T + kTopkWarps - 1) / kTopkWarps;
+  const cudaError_t le_ =
+      L.nsplit > 8 ? launch_k(router_topk_kernel<true>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
+                              L.nsplit, d.k, idx, w, masks)
+                   : launch_k(router_topk_kernel<false>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
+                              L.nsplit, d.k, idx, w, masks);
   return ls_.done(le_);
 }
 

@@ -205,6 +205,11 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const __g
 // One warp per token: sum the split partials in split order, add the bias,
 // pick the k largest (ties: lower index), softmax over them, set the token's
 // bits in the expert bitmasks. Lane l holds experts l, l+32, l+64, l+96.
+// ALL_SPLITS (small batches, many splits of the router's reduction): every
+// split's loads are in flight at once, one memory round trip instead of one
+// per four splits; large batches keep the leaner loop, whose lower register
+// count keeps more token warps resident. The sum order is the same.
+template <bool ALL_SPLITS>
 __global__ void __launch_bounds__(kTopkWarps * 32) router_topk_kernel(const float* __restrict__ partial,
                                                                      const float* __restrict__ bias, int T, int E,
                                                                      int nsplit, int k, int32_t* __restrict__ idx,
@@ -220,6 +225,22 @@ __global__ void __launch_bounds__(kTopkWarps * 32) router_topk_kernel(const floa
   const size_t split_stride = static_cast<size_t>(T) * E;
   const float* base = partial + static_cast<size_t>(t) * E;
   int sp = 0;
+  if (ALL_SPLITS) {
+    float v[kMaxRouterSplits][4];
+#pragma unroll
+    for (int s = 0; s < kMaxRouterSplits; ++s)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = lane + 32 * q;
+        v[s][q] = (s < nsplit && e < E) ? __ldg(base + s * split_stride + e) : 0.f;
+      }
+#pragma unroll
+    for (int s = 0; s < kMaxRouterSplits; ++s)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (s < nsplit) l[q] += v[s][q];
+    sp = nsplit;
+  }
   for (; sp + 4 <= nsplit; sp += 4) {  // four splits' loads in flight, summed in order
     float v[4][4];
 #pragma unroll
