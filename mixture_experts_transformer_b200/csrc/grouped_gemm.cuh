@@ -83,6 +83,16 @@ struct GemmParams {
   CUtensorMap tmA[2];   // [a_rows, K] bf16, box 64 x 128
   CUtensorMap tmB0[2];  // [groups, K, N] bf16, box 64 x 64 x 1 (gate, or the only B)
   CUtensorMap tmB1[2];  // [groups, K, N] bf16 (up; GATEUP only)
+  // Wide boxes: fewer copy instructions per stage for the same bytes.
+  // tmA2: box 64 x 256, the two consecutive 128-row blocks of a paired tile
+  // (a_wide). tmBw0 / tmBw1: B viewed as [groups][N / 64][K][64] (64-column
+  // chunks as a dimension), box 64 x 64 x bw_chunks x 1: bw_chunks adjacent
+  // chunks in one copy, landing 8 KB apart as the per-chunk copies do.
+  CUtensorMap tmA2[2];
+  CUtensorMap tmBw0[2];
+  CUtensorMap tmBw1[2];
+  int a_wide;
+  int bw_chunks;  // 0: per-chunk copies only
   GemmProblem prob[2];
   int nprob;
   // 1: every weight tile is read by one row block (small batches), so B loads
@@ -147,6 +157,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       tma_prefetch_desc(&P.tmA[p]);
       tma_prefetch_desc(&P.tmB0[p]);
       if (GATEUP) tma_prefetch_desc(&P.tmB1[p]);
+      if (PAIRED && P.a_wide) tma_prefetch_desc(&P.tmA2[p]);
+      if (P.bw_chunks) {
+        tma_prefetch_desc(&P.tmBw0[p]);
+        if (GATEUP) tma_prefetch_desc(&P.tmBw1[p]);
+      }
     }
   }
   if (warp == 1) {
@@ -225,17 +240,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           break;
         }
         if (lane == 0) {
-          tma_load_2d(sA + s * kAS, &P.tmA[p], &full[s], kb * kBK, tile.row0);
-          if (has1) tma_load_2d(sA + s * kAS + kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row1);
-          for (int c = 0; c < nch; ++c) {
-            const bool up = GATEUP && c >= cpp;
-            const int col = tile.n0 + (up ? c - cpp : c) * 64;
-            void* dst = sB + s * kBStageBytes + c * kBChunkBytes;
-            const CUtensorMap* mb = up ? &P.tmB1[p] : &P.tmB0[p];
-            if (P.stream_weights)
-              tma_load_3d_hint(dst, mb, &full[s], col, kb * kBK, g, wpol);
-            else
-              tma_load_3d(dst, mb, &full[s], col, kb * kBK, g);
+          if (has1 && P.a_wide && tile.row1 == tile.row0 + kBM) {
+            tma_load_2d(sA + s * kAS, &P.tmA2[p], &full[s], kb * kBK, tile.row0);  // both 128-row blocks
+          } else {
+            tma_load_2d(sA + s * kAS, &P.tmA[p], &full[s], kb * kBK, tile.row0);
+            if (has1) tma_load_2d(sA + s * kAS + kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row1);
+          }
+          if (P.bw_chunks == cpp) {
+            // each projection's cpp chunks in one copy (gate, then up at chunk cpp)
+            for (int q = 0; q < (GATEUP ? 2 : 1); ++q) {
+              void* dst = sB + s * kBStageBytes + q * cpp * kBChunkBytes;
+              const CUtensorMap* mb = q ? &P.tmBw1[p] : &P.tmBw0[p];
+              if (P.stream_weights)
+                tma_load_4d_hint(dst, mb, &full[s], 0, kb * kBK, tile.n0 / 64, g, wpol);
+              else
+                tma_load_4d(dst, mb, &full[s], 0, kb * kBK, tile.n0 / 64, g);
+            }
+          } else {
+            for (int c = 0; c < nch; ++c) {
+              const bool up = GATEUP && c >= cpp;
+              const int col = tile.n0 + (up ? c - cpp : c) * 64;
+              void* dst = sB + s * kBStageBytes + c * kBChunkBytes;
+              const CUtensorMap* mb = up ? &P.tmB1[p] : &P.tmB0[p];
+              if (P.stream_weights)
+                tma_load_3d_hint(dst, mb, &full[s], col, kb * kBK, g, wpol);
+              else
+                tma_load_3d(dst, mb, &full[s], col, kb * kBK, g);
+            }
           }
         }
         ++issued;

@@ -72,6 +72,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tma_prefetch_desc(&P.tmA[p]);
       tma_prefetch_desc(&P.tmB0[p]);
       if (GATEUP) tma_prefetch_desc(&P.tmB1[p]);
+      if (P.bw_chunks) {
+        tma_prefetch_desc(&P.tmBw0[p]);
+        if (GATEUP) tma_prefetch_desc(&P.tmBw1[p]);
+      }
     }
   }
   if (warp == 1) {
@@ -127,11 +131,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[s], both);
           const uint32_t bar = full_even + 8u * s;
           if (my_a) tma_load_2d_pair(sA + s * kP2AStage, &P.tmA[p], bar, kb * kBK, row);
-          for (int c = 0; c < nch; ++c)
+          if (P.bw_chunks == nch) {  // this CTA's chunks in one copy
+            const CUtensorMap* mw = (GATEUP && !leader) ? &P.tmBw1[p] : &P.tmBw0[p];
             if (P.stream_weights)
-              tma_load_3d_pair_hint(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g, wpol);
+              tma_load_4d_pair_hint(sB + s * kP2BStage, mw, bar, 0, kb * kBK, col0 / 64, g, wpol);
             else
-              tma_load_3d_pair(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g);
+              tma_load_4d_pair(sB + s * kP2BStage, mw, bar, 0, kb * kBK, col0 / 64, g);
+          } else {
+            for (int c = 0; c < nch; ++c)
+              if (P.stream_weights)
+                tma_load_3d_pair_hint(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g,
+                                      wpol);
+              else
+                tma_load_3d_pair(sB + s * kP2BStage + c * kBChunkBytes, mb, bar, col0 + c * 64, kb * kBK, g);
+          }
           ++issued;
           if (++s == kP2Stages) {
             s = 0;

@@ -264,6 +264,31 @@ bool map_3d(CUtensorMap* m, const void* base, uint64_t groups, uint64_t K, uint6
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [groups, K, N] bf16 viewed as [groups][N / 64][K][64]: 64-column chunks as a
+// dimension of their own, so one box of 64 x 64 x chunks x 1 brings `chunks`
+// adjacent chunks, each landing as the 64 x 64 box of map_3d would (8 KB
+// apart). Requires N % 64 == 0.
+bool map_4d_chunks(CUtensorMap* m, const void* base, uint64_t groups, uint64_t K, uint64_t N, uint32_t chunks) {
+  const cuuint64_t dims[4] = {64, K, N / 64, groups};
+  const cuuint64_t strides[3] = {N * 2, 128, K * N * 2};
+  const cuuint32_t box[4] = {64, 64, chunks, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The wide boxes of a GEMM (GemmParams::tmA2 / tmBw*): A pairs of 128-row
+// blocks when a_wide, B chunks of `chunks` when nonzero. A map that cannot be
+// encoded leaves the per-block / per-chunk copies in use.
+void set_wide_maps(GemmParams* g, int p, const void* a, uint64_t a_rows, uint64_t K, bool a_wide, const void* b0,
+                   const void* b1, uint64_t groups, uint64_t N, uint32_t chunks) {
+  if (a_wide && !map_2d(&g->tmA2[p], a, a_rows, K, 2 * kBM)) g->a_wide = 0;
+  if (chunks && (!map_4d_chunks(&g->tmBw0[p], b0, groups, K, N, chunks) ||
+                 (b1 && !map_4d_chunks(&g->tmBw1[p], b1, groups, K, N, chunks))))
+    g->bw_chunks = 0;
+}
+
 // Kernel ids of the per-kernel timing records.
 enum KernelId : int {
   kKRouterLogits = 0,
@@ -497,6 +522,10 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   gu.prob[1] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
   gu.nprob = 2;
   gu.stream_weights = stream_weights(d) ? 1 : 0;
+  gu.a_wide = paired_gateup(d) ? 1 : 0;
+  gu.bw_chunks = 2;  // 128 output columns of each projection
+  set_wide_maps(&gu, 0, x_perm, R, d.D, gu.a_wide, p->wg, p->wu, d.E, d.F, 2);
+  set_wide_maps(&gu, 1, xin, d.T, d.D, gu.a_wide, p->sg, p->su, 1, d.S, 2);
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
   gu.next_tile = &counts->next_gateup;
@@ -522,6 +551,11 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   dn.prob[1] = GemmProblem{d.S, d.D, 1, d.T, sbuf, d.D, 1};
   dn.nprob = 2;
   dn.stream_weights = gu.stream_weights;
+  // 256-column tiles: 4 chunks per copy on one SM, 2 per CTA on SM pairs
+  dn.bw_chunks = pair_sm(d, s) ? 2 : 4;
+  dn.a_wide = paired_down(d) && !pair_sm(d, s) ? 1 : 0;
+  set_wide_maps(&dn, 0, h, R, d.F, dn.a_wide, p->wd, nullptr, d.E, d.D, dn.bw_chunks);
+  set_wide_maps(&dn, 1, hs, d.T, d.S, dn.a_wide, p->sd, nullptr, 1, d.D, dn.bw_chunks);
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
   dn.next_tile = &counts->next_down;
@@ -886,6 +920,9 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   gu.prob[0] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
   gu.nprob = 1;
   gu.stream_weights = d.T <= kBM ? 1 : 0;  // one row block reads each weight tile once
+  gu.a_wide = pairs ? 1 : 0;
+  gu.bw_chunks = 2;
+  set_wide_maps(&gu, 0, p->x, d.T, d.D, gu.a_wide, p->wg, p->wu, 1, d.S, 2);
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
   gu.next_tile = &counts->next_gateup;
@@ -911,6 +948,8 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
                            d.D, (split || p->out_f32) ? 1 : 0, static_cast<long long>(d.T) * d.D};
   dn.nprob = 1;
   dn.stream_weights = gu.stream_weights;
+  dn.bw_chunks = pair_dn ? 2 : 4;
+  set_wide_maps(&dn, 0, hs, d.T, d.S, 0, p->wd, nullptr, 1, d.D, dn.bw_chunks);
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
   dn.next_tile = &counts->next_down;
