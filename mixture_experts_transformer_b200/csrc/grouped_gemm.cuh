@@ -43,6 +43,8 @@ constexpr int kStages = 4;
 constexpr int kAStageBytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBChunkBytes = kBK * 64 * 2;    // 8 KB: 64 K-rows x 64 N-columns
 constexpr int kMaxBChunks = 4;
+constexpr int kASmallRows = 32;                  // rows of the small A box
+constexpr int kASmallBytes = kASmallRows * kBK * 2;  // 4 KB
 constexpr int kBStageBytes = kMaxBChunks * kBChunkBytes;
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
@@ -91,7 +93,13 @@ struct GemmParams {
   CUtensorMap tmA2[2];
   CUtensorMap tmBw0[2];
   CUtensorMap tmBw1[2];
+  // tmAs: box 64 x 32 (a_small): a tile of at most 32 rows (small batches
+  // spread over many experts) copies only those; the other 96 rows of its A
+  // stage are left as they are, and the accumulator rows they feed are never
+  // stored.
+  CUtensorMap tmAs[2];
   int a_wide;
+  int a_small;
   int bw_chunks;  // 0: per-chunk copies only
   GemmProblem prob[2];
   int nprob;
@@ -158,6 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       tma_prefetch_desc(&P.tmB0[p]);
       if (GATEUP) tma_prefetch_desc(&P.tmB1[p]);
       if (PAIRED && P.a_wide) tma_prefetch_desc(&P.tmA2[p]);
+      if (P.a_small) tma_prefetch_desc(&P.tmAs[p]);
       if (P.bw_chunks) {
         tma_prefetch_desc(&P.tmBw0[p]);
         if (GATEUP) tma_prefetch_desc(&P.tmBw1[p]);
@@ -226,7 +235,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const int wn = tile_cols<GATEUP>(pr, tile.n0);
       const int cpp = wn >> 6;  // 64-column chunks per projection
       const int nch = GATEUP ? 2 * cpp : cpp;
-      const uint32_t bytes = (has1 ? 2 : 1) * kAStageBytes + nch * kBChunkBytes;
+      const bool a_small = P.a_small && !has1 && tile.rows <= kASmallRows;
+      const uint32_t bytes = (a_small ? kASmallBytes : (has1 ? 2 : 1) * kAStageBytes) + nch * kBChunkBytes;
       const int kb_end = tile.kbn ? tile.kb0 + tile.kbn : kb_all;
       bool ok = true;
       for (int kb = tile.kb0; kb < kb_end; ++kb) {
@@ -242,6 +252,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         if (lane == 0) {
           if (has1 && P.a_wide && tile.row1 == tile.row0 + kBM) {
             tma_load_2d(sA + s * kAS, &P.tmA2[p], &full[s], kb * kBK, tile.row0);  // both 128-row blocks
+          } else if (a_small) {
+            tma_load_2d(sA + s * kAS, &P.tmAs[p], &full[s], kb * kBK, tile.row0);  // the tile's <= 32 rows
           } else {
             tma_load_2d(sA + s * kAS, &P.tmA[p], &full[s], kb * kBK, tile.row0);
             if (has1) tma_load_2d(sA + s * kAS + kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row1);

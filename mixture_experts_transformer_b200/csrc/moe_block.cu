@@ -284,6 +284,7 @@ bool map_4d_chunks(CUtensorMap* m, const void* base, uint64_t groups, uint64_t K
 void set_wide_maps(GemmParams* g, int p, const void* a, uint64_t a_rows, uint64_t K, bool a_wide, const void* b0,
                    const void* b1, uint64_t groups, uint64_t N, uint32_t chunks) {
   if (a_wide && !map_2d(&g->tmA2[p], a, a_rows, K, 2 * kBM)) g->a_wide = 0;
+  if (g->a_small && !map_2d(&g->tmAs[p], a, a_rows, K, kASmallRows)) g->a_small = 0;
   if (chunks && (!map_4d_chunks(&g->tmBw0[p], b0, groups, K, N, chunks) ||
                  (b1 && !map_4d_chunks(&g->tmBw1[p], b1, groups, K, N, chunks))))
     g->bw_chunks = 0;
@@ -523,6 +524,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   gu.nprob = 2;
   gu.stream_weights = stream_weights(d) ? 1 : 0;
   gu.a_wide = paired_gateup(d) ? 1 : 0;
+  gu.a_small = paired_gateup(d) ? 0 : 1;
   gu.bw_chunks = 2;  // 128 output columns of each projection
   set_wide_maps(&gu, 0, x_perm, R, d.D, gu.a_wide, p->wg, p->wu, d.E, d.F, 2);
   set_wide_maps(&gu, 1, xin, d.T, d.D, gu.a_wide, p->sg, p->su, 1, d.S, 2);
@@ -554,6 +556,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   // 256-column tiles: 4 chunks per copy on one SM, 2 per CTA on SM pairs
   dn.bw_chunks = pair_sm(d, s) ? 2 : 4;
   dn.a_wide = paired_down(d) && !pair_sm(d, s) ? 1 : 0;
+  dn.a_small = (pair_sm(d, s) || paired_down(d)) ? 0 : 1;
   set_wide_maps(&dn, 0, h, R, d.F, dn.a_wide, p->wd, nullptr, d.E, d.D, dn.bw_chunks);
   set_wide_maps(&dn, 1, hs, d.T, d.S, dn.a_wide, p->sd, nullptr, 1, d.D, dn.bw_chunks);
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
@@ -608,11 +611,12 @@ bool map_2d_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [groups, rows, cols] bytes; box 128 bytes x 128 rows x 1; 128-byte swizzle.
-bool map_3d_u8(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols) {
+// [groups, rows, cols] bytes; box 128 bytes x box_rows x 1; 128-byte swizzle.
+bool map_3d_u8(CUtensorMap* m, const void* base, uint64_t groups, uint64_t rows, uint64_t cols,
+               uint32_t box_rows = 128) {
   const cuuint64_t dims[3] = {cols, rows, groups};
   const cuuint64_t strides[2] = {cols, rows * cols};
-  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t box[3] = {128, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -769,7 +773,8 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   Fp4Params dn;
   std::memset(&dn, 0, sizeof(dn));
   ok = map_2d_u8(&dn.tmA[0], ws + F.hq, rp, d.F / 2) && map_3d_u8(&dn.tmB0[0], p->wd.q, d.E, d.D, d.F / 2) &&
-       map_2d_u8(&dn.tmA[1], ws + F.hsq, tp, d.S / 2) && map_3d_u8(&dn.tmB0[1], p->sd.q, 1, d.D, d.S / 2);
+       map_2d_u8(&dn.tmA[1], ws + F.hsq, tp, d.S / 2) && map_3d_u8(&dn.tmB0[1], p->sd.q, 1, d.D, d.S / 2) &&
+       map_3d_u8(&dn.tmBw[0], p->wd.q, d.E, d.D, d.F / 2, 256) && map_3d_u8(&dn.tmBw[1], p->sd.q, 1, d.D, d.S / 2, 256);
   if (!ok) return MOE_ERR_CUDA;
   dn.tmB1[0] = dn.tmB0[0];
   dn.tmB1[1] = dn.tmB0[1];
@@ -921,6 +926,7 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   gu.nprob = 1;
   gu.stream_weights = d.T <= kBM ? 1 : 0;  // one row block reads each weight tile once
   gu.a_wide = pairs ? 1 : 0;
+  gu.a_small = pairs ? 0 : 1;
   gu.bw_chunks = 2;
   set_wide_maps(&gu, 0, p->x, d.T, d.D, gu.a_wide, p->wg, p->wu, 1, d.S, 2);
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
@@ -949,6 +955,7 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   dn.nprob = 1;
   dn.stream_weights = gu.stream_weights;
   dn.bw_chunks = pair_dn ? 2 : 4;
+  dn.a_small = pair_dn ? 0 : 1;
   set_wide_maps(&dn, 0, hs, d.T, d.S, 0, p->wd, nullptr, 1, d.D, dn.bw_chunks);
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;

@@ -272,6 +272,7 @@ struct Fp4Params {
   CUtensorMap tmA[2];   // codes [a_rows][K/2] u8, box 128 x 128, 128-byte swizzle
   CUtensorMap tmB0[2];  // codes [groups][N][K/2] u8, box 128 x 128 x 1
   CUtensorMap tmB1[2];
+  CUtensorMap tmBw[2];  // down: the same codes, box 128 x 256 x 1 (both 128-row halves of a tile in one copy)
   Fp4Problem prob[2];
   int nprob;
   const Tile* tiles;
@@ -426,12 +427,11 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
           const uint32_t bytes = kF4ABytes + (two_b ? 2 : 1) * (kF4BBytes / 2) + sf_bytes * (two_b ? 3 : 2);
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(sA + s * kF4ABytes, &P.tmA[p], &full[s], ks * 128, tile.row0);
-          tma_load_3d(sB + s * kF4BBytes, &P.tmB0[p], &full[s], ks * 128, tile.n0, g);
-          if (two_b) {
-            if (GATEUP)
-              tma_load_3d(sB + s * kF4BBytes + kF4BBytes / 2, &P.tmB1[p], &full[s], ks * 128, tile.n0, g);
-            else
-              tma_load_3d(sB + s * kF4BBytes + kF4BBytes / 2, &P.tmB0[p], &full[s], ks * 128, tile.n0 + 128, g);
+          if (!GATEUP && two_b) {
+            tma_load_3d(sB + s * kF4BBytes, &P.tmBw[p], &full[s], ks * 128, tile.n0, g);  // 256 rows
+          } else {
+            tma_load_3d(sB + s * kF4BBytes, &P.tmB0[p], &full[s], ks * 128, tile.n0, g);
+            if (two_b) tma_load_3d(sB + s * kF4BBytes + kF4BBytes / 2, &P.tmB1[p], &full[s], ks * 128, tile.n0, g);
           }
           bulk_load(sSfA + s * kF4SfBytes, sfa + static_cast<size_t>(4 * ks) * 512, sf_bytes, &full[s]);
           bulk_load(sSfB + (2 * s) * kF4SfBytes, sfb0 + static_cast<size_t>(4 * ks) * 512, sf_bytes, &full[s]);
