@@ -10,7 +10,14 @@
 // an MN-major operand, so no weight is repacked.
 //
 // Roles (320 threads, one CTA per SM):
-//   warp 0      TMA producer: A tile 128x64 and B chunks 64(K)x64(N) per stage
+//   warp 0      TMA producer: A tile 128x64 and B chunks 64(K)x64(N) per stage,
+//               in as few copies as the tile allows (one 256-row box for the
+//               two row blocks of a paired tile, a 32-row box for a tile of at
+//               most 32 rows, one box for all of a projection's chunks through
+//               a 4-D view of B): measured, the copy count per stage matters as
+//               much as the bytes. Small batches stream B with an L2
+//               evict-first policy (each weight tile is read by one row block).
+//               A tile may cover a K range only (split-K partial sums).
 //   warp 1      MMA issuer (one thread): 4 x tcgen05.mma (K = 16) per stage
 //   warps 2..9  epilogue, two warps per TMEM lane quarter (each half of the
 //               column chunks): tcgen05.ld the fp32 accumulator, apply GeGLU
