@@ -766,7 +766,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   {
     LaunchScope ls_(kKFp4GateUp, st);
     const cudaError_t le_ =
-        launch_k(fp4_gemm_kernel<true>, std::min(s->sm_count, L.max_tiles_gu), kF4Threads, kF4SmemBytes, st, gu);
+        launch_k(fp4_gemm_kernel<true>, std::min(s->sm_count, L.max_tiles_gu), f4_threads<true>(), kF4SmemBytes, st, gu);
     MOE_TRY(ls_.done(le_));
   }
 
@@ -790,7 +790,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   {
     LaunchScope ls_(kKFp4Down, st);
     const cudaError_t le_ =
-        launch_k(fp4_gemm_kernel<false>, std::min(s->sm_count, L.max_tiles_dn), kF4Threads, kF4SmemBytes, st, dn);
+        launch_k(fp4_gemm_kernel<false>, std::min(s->sm_count, L.max_tiles_dn), f4_threads<false>(), kF4SmemBytes, st, dn);
     MOE_TRY(ls_.done(le_));
   }
   {

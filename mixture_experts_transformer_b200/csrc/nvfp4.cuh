@@ -247,6 +247,14 @@ constexpr int kF4SfBytes = 4 * 512;              // 4 atoms (4 x 64 K) of one 12
 constexpr int kF4Stages = 4;
 constexpr int kF4SfSlots = 16;                   // TMEM scale slots (ring over 64-K steps)
 constexpr int kF4Threads = 320;                  // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
+// The gate|up GEMM adds 4 scale warps (see the kernel). Measured at T=2048:
+// gate|up 122 -> 98 us with them; the down GEMM keeps copying the scales from
+// its MMA thread, since at 448 threads its epilogue (128 accumulator values
+// per thread held in registers) spills: 80 -> 137 us.
+template <bool GATEUP>
+__host__ __device__ constexpr int f4_threads() {
+  return GATEUP ? kF4Threads + 128 : kF4Threads;
+}
 constexpr int kF4StgWarpBytes = 1024;            // epilogue staging per warp (32 rows x 32 B)
 constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 8 * kF4StgWarpBytes + 1024 + 256;
 
@@ -299,6 +307,15 @@ __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
   return d;
 }
 
+// 4 consecutive 32-bit TMEM columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
@@ -336,7 +353,7 @@ __device__ __forceinline__ int f4_tile_cols(const Fp4Problem& pr, int n0) {
 // once. From 256: scale slots, slot i holding the A scales at +0, B block 0 at
 // +4, B block 1 at +8.
 template <bool GATEUP>
-__global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_constant__ Fp4Params P) {
+__global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const __grid_constant__ Fp4Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -351,7 +368,8 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
   uint64_t* acc_full = empty + kF4Stages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_ready = drain + 1;  // a stage's scale atoms are in TMEM (one arrival per scale warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_ready + kF4Stages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -360,6 +378,7 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
     for (int s = 0; s < kF4Stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 4);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
@@ -484,18 +503,26 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
             ok = false;
             break;
           }
+          // gate|up: the stage's scale atoms are written into TMEM by the
+          // scale warps (tcgen05.st), off this thread's MMA stream
+          if (GATEUP && !mbar_wait(&sf_ready[s], ph, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
           tc_fence_after_sync();
           const int nks = min(4, k64 - 4 * ks);
           const uint32_t a_addr = smem_u32(sA + s * kF4ABytes);
           const uint32_t b_addr = smem_u32(sB + s * kF4BBytes);
-          const uint32_t sfa_addr = smem_u32(sSfA + s * kF4SfBytes);
-          const uint32_t sfb_addr = smem_u32(sSfB + (2 * s) * kF4SfBytes);
-          // the whole stage's scale atoms first (the copies pipeline), then its MMAs
-          for (int i = 0; i < nks; ++i) {
-            const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
-            tmem_cp_32x128b_x4(cols, sdesc_sf_atom(sfa_addr + i * 512));
-            tmem_cp_32x128b_x4(cols + 4, sdesc_sf_atom(sfb_addr + i * 512));
-            if (two_b) tmem_cp_32x128b_x4(cols + 8, sdesc_sf_atom(sfb_addr + kF4SfBytes + i * 512));
+          if (!GATEUP) {
+            // down: the whole stage's scale atoms first (the copies pipeline), then its MMAs
+            const uint32_t sfa_addr = smem_u32(sSfA + s * kF4SfBytes);
+            const uint32_t sfb_addr = smem_u32(sSfB + (2 * s) * kF4SfBytes);
+            for (int i = 0; i < nks; ++i) {
+              const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
+              tmem_cp_32x128b_x4(cols, sdesc_sf_atom(sfa_addr + i * 512));
+              tmem_cp_32x128b_x4(cols + 4, sdesc_sf_atom(sfb_addr + i * 512));
+              if (two_b) tmem_cp_32x128b_x4(cols + 8, sdesc_sf_atom(sfb_addr + kF4SfBytes + i * 512));
+            }
           }
           for (int i = 0; i < nks; ++i) {
             const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
@@ -528,6 +555,56 @@ __global__ void __launch_bounds__(kF4Threads, 1) fp4_gemm_kernel(const __grid_co
         uint32_t dummy = 0;
         mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), P.err);
       }
+    }
+  } else if (GATEUP && warp >= 10) {
+    // ------------------------------------------------------- scale warps
+    // Warps 10..13 (TMEM lane quarters 2, 3, 0, 1): for every stage, in the
+    // MMA thread's order, each writes its quarter of the stage's scale atoms
+    // into the TMEM slots the MMAs read. An atom (512 B) holds 32 rows of
+    // 16 B; row i goes to columns c..c+3 of lane 32 q + i in every quarter q,
+    // the layout tcgen05.cp .32x128b.warpx4 would produce, but from the
+    // warps' registers, so the tensor pipe runs only MMAs. A slot is rewritten
+    // only after full[] of its stage completed, i.e. after the MMAs that read
+    // its previous contents (four stages back) have finished.
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int s = 0, slot = 0;
+    uint32_t ph = 0;
+    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      const Tile tile = P.tiles[ti];
+      const int p = tile.pg >> 16;
+      if (p >= P.nprob) break;
+      const Fp4Problem& pr = P.prob[p];
+      const int k64 = pr.K / 64;
+      const int nstage = (pr.K + kF4KStage - 1) / kF4KStage;
+      const bool two_b = GATEUP || (tile.n0 + 128 < pr.N);
+      bool ok = true;
+      for (int ks = 0; ks < nstage; ++ks) {
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&full[s], ph, abort_flag, P.err);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        const int nks = min(4, k64 - 4 * ks);
+        const uint8_t* sfa = sSfA + s * kF4SfBytes + lane * 16;
+        const uint8_t* sfb = sSfB + (2 * s) * kF4SfBytes + lane * 16;
+        for (int i = 0; i < nks; ++i) {
+          const uint32_t cols = tmem_base + lane_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
+          tmem_st_32x32b_x4(cols, *reinterpret_cast<const uint4*>(sfa + i * 512));
+          tmem_st_32x32b_x4(cols + 4, *reinterpret_cast<const uint4*>(sfb + i * 512));
+          if (two_b) tmem_st_32x32b_x4(cols + 8, *reinterpret_cast<const uint4*>(sfb + kF4SfBytes + i * 512));
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready[s]);
+        slot = (slot + nks) % kF4SfSlots;
+        if (++s == kF4Stages) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+      if (!ok) break;
     }
   } else {
     // ----------------------------------------------------------- epilogue
