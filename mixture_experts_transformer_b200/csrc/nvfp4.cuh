@@ -247,13 +247,11 @@ constexpr int kF4SfBytes = 4 * 512;              // 4 atoms (4 x 64 K) of one 12
 constexpr int kF4Stages = 4;
 constexpr int kF4SfSlots = 16;                   // TMEM scale slots (ring over 64-K steps)
 constexpr int kF4Threads = 320;                  // producer, MMA, 8 epilogue warps (2 per TMEM lane quarter)
-// The gate|up GEMM adds 4 scale warps (see the kernel). Measured at T=2048:
-// gate|up 122 -> 98 us with them; the down GEMM keeps copying the scales from
-// its MMA thread, since at 448 threads its epilogue (128 accumulator values
-// per thread held in registers) spills: 80 -> 137 us.
+// Both GEMMs add 4 scale warps (see the kernel): measured at T=2048, gate|up
+// 122 -> 98 us with them.
 template <bool GATEUP>
 __host__ __device__ constexpr int f4_threads() {
-  return GATEUP ? kF4Threads + 128 : kF4Threads;
+  return kF4Threads + 128;
 }
 constexpr int kF4StgWarpBytes = 1024;            // epilogue staging per warp (32 rows x 32 B)
 constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 8 * kF4StgWarpBytes + 1024 + 256;
@@ -503,9 +501,9 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
             ok = false;
             break;
           }
-          // gate|up: the stage's scale atoms are written into TMEM by the
-          // scale warps (tcgen05.st), off this thread's MMA stream
-          if (GATEUP && !mbar_wait(&sf_ready[s], ph, abort_flag, P.err)) {
+          // the stage's scale atoms are written into TMEM by the scale warps
+          // (tcgen05.st), off this thread's MMA stream
+          if (!mbar_wait(&sf_ready[s], ph, abort_flag, P.err)) {
             ok = false;
             break;
           }
@@ -513,17 +511,6 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
           const int nks = min(4, k64 - 4 * ks);
           const uint32_t a_addr = smem_u32(sA + s * kF4ABytes);
           const uint32_t b_addr = smem_u32(sB + s * kF4BBytes);
-          if (!GATEUP) {
-            // down: the whole stage's scale atoms first (the copies pipeline), then its MMAs
-            const uint32_t sfa_addr = smem_u32(sSfA + s * kF4SfBytes);
-            const uint32_t sfb_addr = smem_u32(sSfB + (2 * s) * kF4SfBytes);
-            for (int i = 0; i < nks; ++i) {
-              const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
-              tmem_cp_32x128b_x4(cols, sdesc_sf_atom(sfa_addr + i * 512));
-              tmem_cp_32x128b_x4(cols + 4, sdesc_sf_atom(sfb_addr + i * 512));
-              if (two_b) tmem_cp_32x128b_x4(cols + 8, sdesc_sf_atom(sfb_addr + kF4SfBytes + i * 512));
-            }
-          }
           for (int i = 0; i < nks; ++i) {
             const uint32_t cols = tmem_base + kAccCols + ((slot + i) % kF4SfSlots) * 16;
             // 64 K of e2m1 = 32 B per row inside the 128-byte swizzled rows
@@ -556,7 +543,7 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
         mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), P.err);
       }
     }
-  } else if (GATEUP && warp >= 10) {
+  } else if (warp >= 10) {
     // ------------------------------------------------------- scale warps
     // Warps 10..13 (TMEM lane quarters 2, 3, 0, 1): for every stage, in the
     // MMA thread's order, each writes its quarter of the stage's scale atoms
@@ -627,25 +614,33 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
       const uint32_t tbase = tmem_base + acc_i * kAccStride + (static_cast<uint32_t>(quarter * 32) << 16);
       const bool valid = r < tile.rows;
       const int grow = tile.row0 + r;
-      // Bring this thread's accumulator columns into registers and hand TMEM
-      // back at once, so the next tile's MMAs overlap the math and stores below.
       // Column chunks of 32: j = half * 32 + 64 c (c = 0..3 while j < wn).
+      // Gate|up brings all of this thread's accumulator columns (gate and up
+      // of chunks 0, 1) into registers and hands TMEM back at once, so the
+      // next tile's MMAs overlap the math and stores below. Down holds 4
+      // chunks: chunks 0, 1 are converted and stored first, then chunks 2, 3
+      // are loaded and TMEM handed back (64 values in registers at a time).
       uint32_t acc[4][32];
-#pragma unroll
-      for (int c = 0; c < (GATEUP ? 2 : 4); ++c) {
-        const int j = half * 32 + 64 * c;
-        if (j < wn) {
-          tmem_ld_32x32b_x32(tbase + j, acc[c]);
-          if (GATEUP) tmem_ld_32x32b_x32(tbase + 128 + j, acc[2 + c]);
+      auto release_acc = [&]() {
+        tmem_ld_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc_i]);
+        if (++acc_i == kAccStages) {
+          acc_i = 0;
+          acc_ph ^= 1;
         }
-      }
-      tmem_ld_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc_i]);
-      if (++acc_i == kAccStages) {
-        acc_i = 0;
-        acc_ph ^= 1;
+      };
+      if (GATEUP) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int j = half * 32 + 64 * c;
+          if (j < wn) {
+            tmem_ld_32x32b_x32(tbase + j, acc[c]);
+            tmem_ld_32x32b_x32(tbase + 128 + j, acc[2 + c]);
+          }
+        }
+        release_acc();
       }
       if (GATEUP) {
         const float ag = 1.0f / (pr.ga * pr.gb0[g]);
@@ -682,8 +677,18 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int j = half * 32 + 64 * c;
+          if ((c & 1) == 0) {  // load chunks c, c + 1; after the second pair TMEM is no longer needed
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+              if (j + 64 * u < wn) tmem_ld_32x32b_x32(tbase + j + 64 * u, acc[u]);
+            if (c == 2) {
+              release_acc();
+            } else {
+              tmem_ld_wait();
+            }
+          }
           if (j >= wn) continue;
-          uint32_t* a = acc[c];
+          uint32_t* a = acc[c & 1];
           if (pr.out_f32) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
