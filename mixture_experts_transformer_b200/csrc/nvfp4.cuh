@@ -20,13 +20,14 @@
 //
 // The GEMM (fp4_gemm_kernel) is the bf16 grouped GEMM's structure with
 // `tcgen05.mma.kind::mxf4nvf4.block_scale.block16`: TMA brings 256-K stages of
-// A and B codes plus the matching scale atoms (a bulk copy); per stage the MMA
-// thread first moves all of the stage's scale atoms into TMEM with tcgen05.cp
-// (32x128b, broadcast to the four lane quarters; the copies pipeline), then
-// issues two M=128, N=128 MMAs per 64-K step. Eight epilogue warps (two per
-// TMEM lane quarter, each half of the columns) multiply by 1/(G_act *
-// G_weight); the gate|up epilogue then quantises the GeGLU rows h to NVFP4 for
-// the down projection.
+// A and B codes plus the matching scale atoms (a bulk copy); four scale warps
+// write each stage's atoms into TMEM from their registers (tcgen05.st, each
+// atom row replicated to the four lane quarters), so the MMA thread's tensor
+// stream holds only the MMAs: one M=128, N=256 MMA per 64-K step covering
+// both 128-column halves of the tile. Eight epilogue warps (two per TMEM lane
+// quarter, each half of the columns) multiply by 1/(G_act * G_weight); the
+// gate|up epilogue then quantises the GeGLU rows h to NVFP4 for the down
+// projection.
 #pragma once
 
 #include "grouped_gemm.cuh"
@@ -295,16 +296,6 @@ __host__ __device__ constexpr uint32_t idesc_nvf4_m128(int n) {
          | (static_cast<uint32_t>(128 >> 4) << 24);   // M / 16
 }
 
-// Shared-memory descriptor of one 512-byte scale atom for tcgen05.cp
-// (no swizzle, K-major: 8-row groups of 16-byte rows, 128 bytes apart).
-__device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>(128 >> 4) << 32;  // stride byte offset
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;
-}
-
 // 4 consecutive 32-bit TMEM columns of this warp's 32 lanes from registers.
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
@@ -314,9 +305,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 
 __device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
