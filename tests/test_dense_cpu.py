@@ -70,3 +70,22 @@ def test_dense_host_validation(lib):
     assert lib.moe_dense_ffn_forward(None, None) == B.MOE_ERR_INVALID_ARG
     p = B.make_dense_params(64)
     assert B.moe_dense_workspace_bytes(p) >= 64 * inputs.E4B_HIDDEN_DIM * 2
+
+
+def test_dense_workspace_holds_split_k_partials(lib):
+    """Small batches cut the down GEMM's reduction into K ranges whose fp32
+    partial sums live in the workspace (about one wave of (column tile, K
+    range) items at 148 SMs, at least 4 K blocks each): at the E4B decode
+    shape, 10 column tiles of 256 give 14 ranges of 160 K blocks, i.e. 14
+    partial [64, 2560] fp32 planes beyond the bf16 hidden rows. Large batches
+    (T >= 256, paired GEMMs) never split."""
+    D, S = inputs.E4B_EMBED_DIM, inputs.E4B_HIDDEN_DIM
+    dec = B.moe_dense_workspace_bytes(B.make_dense_params(64))
+    assert dec >= 64 * S * 2 + 14 * 64 * D * 4
+    # a hidden dim too short to split (K blocks / 4 < 2) keeps one range
+    small = B.moe_dense_workspace_bytes(B.make_dense_params(64, embed_dim=256, hidden_dim=320))
+    assert small < 64 * 320 * 2 + 2 * 64 * 256 * 4
+    # T = 256 takes the paired kernels: no partial planes at all
+    big = B.moe_dense_workspace_bytes(B.make_dense_params(256))
+    assert big < 256 * S * 2 + 256 * D * 4
+
