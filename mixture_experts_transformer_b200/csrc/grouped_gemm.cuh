@@ -9,8 +9,13 @@
 // N contiguous (the weights exactly as given), which the tensor core reads as
 // an MN-major operand, so no weight is repacked.
 //
-// Roles (320 threads, one CTA per SM):
-//   warp 0      TMA producer: A tile 128x64 and B chunks 64(K)x64(N) per stage,
+// Roles (384 threads, one CTA per SM):
+//   warp 0      TMA producer: schedules the tiles (work counter, tile ring) and,
+//               with warps 10 and 11, issues each stage's copies (copy i of a
+//               stage from thread i % 3: the A rows, the gate chunks, the up
+//               chunks): one thread issues ~2.2 M copies per second however many
+//               are in flight, and more issuing warps scale that (measured).
+//               Per stage: A tile 128x64 and B chunks 64(K)x64(N),
 //               in as few copies as the tile allows (one 256-row box for the
 //               two row blocks of a paired tile, a 32-row box for a tile of at
 //               most 32 rows, one box for all of a projection's chunks through
@@ -56,6 +61,12 @@ constexpr int kBStageBytes = kMaxBChunks * kBChunkBytes;
 constexpr int kAccCols = 256;
 constexpr int kTmemCols = 512;
 constexpr int kGemmThreads = 320;
+// The single-SM grouped GEMM issues a stage's copies from kNProd threads in
+// different warps (warp 0 and warps 10, 11): one thread issues ~2.2 M TMA
+// copies per second however many are in flight, and more issuing warps
+// scale that linearly (measured).
+constexpr int kNProd = 3;
+constexpr int kGemmThreadsSm = kGemmThreads + 32 * (kNProd - 1);
 constexpr int kEpiWarps = 8;
 constexpr int kTileRing = 8;  // tile indices handed from the producer to the MMA and epilogue warps
 constexpr int kStageBytesTotal = kStages * (kAStageBytes + kBStageBytes);
@@ -127,7 +138,7 @@ __device__ __forceinline__ int tile_cols(const GemmProblem& pr, int n0) {
 }
 
 template <bool GATEUP, bool PAIRED = false>
-__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams P) {
+__global__ void __launch_bounds__(kGemmThreadsSm, 1) grouped_gemm_kernel(const __grid_constant__ GemmParams P) {
   constexpr int kSt = PAIRED ? 3 : kStages;
   constexpr int kAS = PAIRED ? 2 * kAStageBytes : kAStageBytes;
   static_assert(kSt * (kAS + kBStageBytes) <= kStages * (kAStageBytes + kBStageBytes), "shared memory budget");
@@ -152,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], kNProd);  // one arrival (with its bytes) per issuing thread
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -162,7 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     mbar_init(drain, 1);
     for (int r = 0; r < kTileRing; ++r) {
       mbar_init(&tile_full[r], 1);
-      mbar_init(&tile_empty[r], 1 + kEpiWarps);  // the MMA thread and every epilogue warp read each index
+      mbar_init(&tile_empty[r], 1 + kEpiWarps + (kNProd - 1));  // MMA thread, epilogue and copy warps read each index
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -193,17 +204,118 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   pdl_wait_then_release();
   const int num_tiles = *P.num_tiles;
 
+  const uint64_t wpol = l2_policy_evict_first();  // streamed weights go before activations
+  // A tile's fields, checked before any copy is addressed from them.
+  auto tile_ok = [&](const Tile& tile) -> bool {
+    const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+    if (p >= P.nprob) return false;
+    const GemmProblem& pr = P.prob[p];
+    const bool has1 = PAIRED && tile.rows1 > 0;
+    const int kb_all = pr.K / kBK;
+    return !(g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || tile.rows < 1 || tile.rows > kBM ||
+             tile.n0 < 0 || tile.n0 >= pr.N || (tile.n0 & 63) ||
+             (has1 && (tile.row1 < 0 || tile.row1 >= pr.a_rows || tile.rows1 > kBM)) || tile.kb0 < 0 ||
+             tile.kbn < 0 || tile.kb0 + (tile.kbn ? tile.kbn : kb_all) > kb_all ||
+             (tile.kbn && (GATEUP || !pr.out_f32 || tile.row1 < 0)));
+  };
+  // The copies of stage st (K block kb) of a tile, in a fixed order: the A
+  // rows, then the B chunks. Copy i belongs to issuing thread i % kNProd;
+  // returns the bytes of thread grp's copies and, with doit, issues them.
+  auto stage_copies = [&](int grp, bool doit, int st, int kb, const Tile& tile) -> uint32_t {
+    const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+    const GemmProblem& pr = P.prob[p];
+    const bool has1 = PAIRED && tile.rows1 > 0;
+    const int wn = tile_cols<GATEUP>(pr, tile.n0);
+    const int cpp = wn >> 6;  // 64-column chunks per projection
+    const int nch = GATEUP ? 2 * cpp : cpp;
+    const bool a_small = P.a_small && !has1 && tile.rows <= kASmallRows;
+    uint32_t bytes = 0;
+    int i = 0;
+    auto mine = [&]() { return (i++ % kNProd) == grp; };
+    if (has1 && P.a_wide && tile.row1 == tile.row0 + kBM) {
+      if (mine()) {  // both 128-row blocks
+        bytes += 2 * kAStageBytes;
+        if (doit) tma_load_2d(sA + st * kAS, &P.tmA2[p], &full[st], kb * kBK, tile.row0);
+      }
+    } else if (a_small) {
+      if (mine()) {  // the tile's <= 32 rows
+        bytes += kASmallBytes;
+        if (doit) tma_load_2d(sA + st * kAS, &P.tmAs[p], &full[st], kb * kBK, tile.row0);
+      }
+    } else {
+      if (mine()) {
+        bytes += kAStageBytes;
+        if (doit) tma_load_2d(sA + st * kAS, &P.tmA[p], &full[st], kb * kBK, tile.row0);
+      }
+      if (has1 && mine()) {
+        bytes += kAStageBytes;
+        if (doit) tma_load_2d(sA + st * kAS + kAStageBytes, &P.tmA[p], &full[st], kb * kBK, tile.row1);
+      }
+    }
+    if (P.bw_chunks == cpp) {
+      // each projection's cpp chunks in one copy (gate, then up at chunk cpp)
+      for (int q = 0; q < (GATEUP ? 2 : 1); ++q) {
+        if (!mine()) continue;
+        bytes += cpp * kBChunkBytes;
+        if (!doit) continue;
+        void* dst = sB + st * kBStageBytes + q * cpp * kBChunkBytes;
+        const CUtensorMap* mb = q ? &P.tmBw1[p] : &P.tmBw0[p];
+        if (P.stream_weights)
+          tma_load_4d_hint(dst, mb, &full[st], 0, kb * kBK, tile.n0 / 64, g, wpol);
+        else
+          tma_load_4d(dst, mb, &full[st], 0, kb * kBK, tile.n0 / 64, g);
+      }
+    } else {
+      for (int c = 0; c < nch; ++c) {
+        if (!mine()) continue;
+        bytes += kBChunkBytes;
+        if (!doit) continue;
+        const bool up = GATEUP && c >= cpp;
+        const int col = tile.n0 + (up ? c - cpp : c) * 64;
+        void* dst = sB + st * kBStageBytes + c * kBChunkBytes;
+        const CUtensorMap* mb = up ? &P.tmB1[p] : &P.tmB0[p];
+        if (P.stream_weights)
+          tma_load_3d_hint(dst, mb, &full[st], col, kb * kBK, g, wpol);
+        else
+          tma_load_3d(dst, mb, &full[st], col, kb * kBK, g);
+      }
+    }
+    return bytes;
+  };
+  // one issuing thread's part of stage st: arm the barrier with its bytes, then copy
+  auto arm_and_copy = [&](int grp, int st, int kb, const Tile& tile) {
+    const uint32_t b = stage_copies(grp, false, st, kb, tile);
+    if (b)
+      mbar_arrive_expect_tx(&full[st], b);
+    else
+      mbar_arrive(&full[st]);
+    stage_copies(grp, true, st, kb, tile);
+  };
+  // after an abort: let this thread's copies in flight land before the CTA's memory goes away
+  auto drain_copies = [&](int s_now, uint32_t ph_now, int issued) {
+    int st = s_now;
+    uint32_t sp = ph_now;
+    const int pending = issued < kSt ? issued : kSt;
+    for (int i = 0; i < pending; ++i) {
+      if (--st < 0) {
+        st = kSt - 1;
+        sp ^= 1;
+      }
+      uint32_t dummy = 0;
+      mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
+    }
+  };
+
   if (warp == 0) {
     // -------------------------------------------------------- TMA producer
     // The whole warp walks the tiles; lane 0 takes the next tile index from
-    // the work counter, publishes it in the tile ring (-1 ends the work), arms
-    // each stage's barrier and issues the loads.
+    // the work counter, publishes it in the tile ring (-1 ends the work), and
+    // issues its share of each stage's copies (copy thread 0).
     int s = 0, issued = 0;
     uint32_t ph = 0;
     int rs = 0;
     uint32_t rph = 0;
     int ti = 0;
-    const uint64_t wpol = l2_policy_evict_first();  // streamed weights go before activations
     if (lane == 0) ti = atomicAdd(P.next_tile, 1);
     ti = __shfl_sync(0xffffffffu, ti, 0);
     while (true) {
@@ -224,69 +336,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       int next = 0;
       if (lane == 0) next = atomicAdd(P.next_tile, 1);  // its latency hides behind this tile's loads
       const Tile tile = P.tiles[ti];
-      const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
-      const bool bad_p = p >= P.nprob;
-      const GemmProblem& pr = P.prob[bad_p ? 0 : p];
-      const bool has1 = PAIRED && tile.rows1 > 0;
-      const int kb_all = pr.K / kBK;
-      if (bad_p || g >= pr.groups || tile.row0 < 0 || tile.row0 >= pr.a_rows || tile.rows < 1 || tile.rows > kBM ||
-          tile.n0 < 0 || tile.n0 >= pr.N || (has1 && (tile.row1 < 0 || tile.row1 >= pr.a_rows || tile.rows1 > kBM)) ||
-          tile.kb0 < 0 || tile.kbn < 0 || tile.kb0 + (tile.kbn ? tile.kbn : kb_all) > kb_all ||
-          (tile.kbn && (GATEUP || !pr.out_f32 || tile.row1 < 0))) {
+      if (!tile_ok(tile)) {
         if (lane == 0) {
           atomicOr(P.err, kErrBadTile);
           *abort_flag = 1;
         }
         break;
       }
-      const int wn = tile_cols<GATEUP>(pr, tile.n0);
-      const int cpp = wn >> 6;  // 64-column chunks per projection
-      const int nch = GATEUP ? 2 * cpp : cpp;
-      const bool a_small = P.a_small && !has1 && tile.rows <= kASmallRows;
-      const uint32_t bytes = (a_small ? kASmallBytes : (has1 ? 2 : 1) * kAStageBytes) + nch * kBChunkBytes;
-      const int kb_end = tile.kbn ? tile.kb0 + tile.kbn : kb_all;
+      const GemmProblem& pr = P.prob[tile.pg >> 16];
+      const int kb_end = tile.kbn ? tile.kb0 + tile.kbn : pr.K / kBK;
       bool ok = true;
       for (int kb = tile.kb0; kb < kb_end; ++kb) {
         int waited = 1;
         if (lane == 0) {
           waited = mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err);
-          if (waited) mbar_arrive_expect_tx(&full[s], bytes);
+          if (waited) arm_and_copy(0, s, kb, tile);
         }
         if (!__shfl_sync(0xffffffffu, waited, 0)) {
           ok = false;
           break;
-        }
-        if (lane == 0) {
-          if (has1 && P.a_wide && tile.row1 == tile.row0 + kBM) {
-            tma_load_2d(sA + s * kAS, &P.tmA2[p], &full[s], kb * kBK, tile.row0);  // both 128-row blocks
-          } else if (a_small) {
-            tma_load_2d(sA + s * kAS, &P.tmAs[p], &full[s], kb * kBK, tile.row0);  // the tile's <= 32 rows
-          } else {
-            tma_load_2d(sA + s * kAS, &P.tmA[p], &full[s], kb * kBK, tile.row0);
-            if (has1) tma_load_2d(sA + s * kAS + kAStageBytes, &P.tmA[p], &full[s], kb * kBK, tile.row1);
-          }
-          if (P.bw_chunks == cpp) {
-            // each projection's cpp chunks in one copy (gate, then up at chunk cpp)
-            for (int q = 0; q < (GATEUP ? 2 : 1); ++q) {
-              void* dst = sB + s * kBStageBytes + q * cpp * kBChunkBytes;
-              const CUtensorMap* mb = q ? &P.tmBw1[p] : &P.tmBw0[p];
-              if (P.stream_weights)
-                tma_load_4d_hint(dst, mb, &full[s], 0, kb * kBK, tile.n0 / 64, g, wpol);
-              else
-                tma_load_4d(dst, mb, &full[s], 0, kb * kBK, tile.n0 / 64, g);
-            }
-          } else {
-            for (int c = 0; c < nch; ++c) {
-              const bool up = GATEUP && c >= cpp;
-              const int col = tile.n0 + (up ? c - cpp : c) * 64;
-              void* dst = sB + s * kBStageBytes + c * kBChunkBytes;
-              const CUtensorMap* mb = up ? &P.tmB1[p] : &P.tmB0[p];
-              if (P.stream_weights)
-                tma_load_3d_hint(dst, mb, &full[s], col, kb * kBK, g, wpol);
-              else
-                tma_load_3d(dst, mb, &full[s], col, kb * kBK, g);
-            }
-          }
         }
         ++issued;
         if (++s == kSt) {
@@ -298,20 +366,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       ti = __shfl_sync(0xffffffffu, next, 0);
     }
     __syncwarp();
-    if (lane == 0 && *abort_flag) {
-      // let copies already in flight land before the CTA's memory goes away
-      int st = s;
-      uint32_t sp = ph;
-      const int pending = issued < kSt ? issued : kSt;
-      for (int i = 0; i < pending; ++i) {
-        if (--st < 0) {
-          st = kSt - 1;
-          sp ^= 1;
-        }
-        uint32_t dummy = 0;
-        mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
-      }
-    }
+    if (lane == 0 && *abort_flag) drain_copies(s, ph, issued);
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
@@ -385,6 +440,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
         uint32_t dummy = 0;
         mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), P.err);
       }
+    }
+  } else if (warp >= 2 + kEpiWarps) {
+    // -------------------------------------------------- copy warps 10, 11
+    // Lane 0 walks the tiles of the ring and issues copy thread grp's share of
+    // every stage (the stage order and barriers of the producer warp).
+    const int grp = warp - (1 + kEpiWarps);  // 1, 2
+    if (lane == 0) {
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      int rs = 0;
+      uint32_t rph = 0;
+      while (true) {
+        if (!mbar_wait(&tile_full[rs], rph, abort_flag, P.err)) break;
+        const int ti = tile_ring[rs];
+        mbar_arrive(&tile_empty[rs]);
+        if (++rs == kTileRing) {
+          rs = 0;
+          rph ^= 1;
+        }
+        if (ti < 0) break;
+        const Tile tile = P.tiles[ti];
+        if (!tile_ok(tile)) break;  // the producer warp reports it
+        const GemmProblem& pr = P.prob[tile.pg >> 16];
+        const int kb_end = tile.kbn ? tile.kb0 + tile.kbn : pr.K / kBK;
+        bool ok = true;
+        for (int kb = tile.kb0; kb < kb_end; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          arm_and_copy(grp, s, kb, tile);
+          ++issued;
+          if (++s == kSt) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) drain_copies(s, ph, issued);
     }
   } else {
     // ----------------------------------------------------------- epilogue

@@ -536,8 +536,8 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   {
   LaunchScope ls_(kKGemmGateUp, st);
   const cudaError_t le_ =
-      paired_gateup(d) ? launch_k(grouped_gemm_kernel<true, true>, grid_gu, kGemmThreads, kGemmSmemBytes, st, gu)
-                       : launch_k(grouped_gemm_kernel<true>, grid_gu, kGemmThreads, kGemmSmemBytes, st, gu);
+      paired_gateup(d) ? launch_k(grouped_gemm_kernel<true, true>, grid_gu, kGemmThreadsSm, kGemmSmemBytes, st, gu)
+                       : launch_k(grouped_gemm_kernel<true>, grid_gu, kGemmThreadsSm, kGemmSmemBytes, st, gu);
   MOE_TRY(ls_.done(le_));
   }
 
@@ -568,8 +568,8 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   LaunchScope ls_(kKGemmDown, st);
   const cudaError_t le_ =
       pair_sm(d, s) ? launch_k(grouped_gemm_pair_kernel<false>, 2 * s->pair_clusters_dn, kGemmThreads, kP2SmemBytes, st, dn)
-      : paired_down(d) ? launch_k(grouped_gemm_kernel<false, true>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn)
-                       : launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreads, kGemmSmemBytes, st, dn);
+      : paired_down(d) ? launch_k(grouped_gemm_kernel<false, true>, grid_dn, kGemmThreadsSm, kGemmSmemBytes, st, dn)
+                       : launch_k(grouped_gemm_kernel<false>, grid_dn, kGemmThreadsSm, kGemmSmemBytes, st, dn);
   MOE_TRY(ls_.done(le_));
   }
 
@@ -936,8 +936,8 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   {
     LaunchScope ls_(kKGemmGateUp, st);
     const int grid = std::min(s->sm_count, L.max_gu);
-    MOE_TRY(ls_.done(pairs ? launch_k(grouped_gemm_kernel<true, true>, grid, kGemmThreads, kGemmSmemBytes, st, gu)
-                           : launch_k(grouped_gemm_kernel<true>, grid, kGemmThreads, kGemmSmemBytes, st, gu)));
+    MOE_TRY(ls_.done(pairs ? launch_k(grouped_gemm_kernel<true, true>, grid, kGemmThreadsSm, kGemmSmemBytes, st, gu)
+                           : launch_k(grouped_gemm_kernel<true>, grid, kGemmThreadsSm, kGemmSmemBytes, st, gu)));
   }
   GemmParams dn;
   std::memset(&dn, 0, sizeof(dn));
@@ -966,7 +966,7 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
     const int grid = std::min(s->sm_count, L.max_dn);
     MOE_TRY(ls_.done(pair_dn ? launch_k(grouped_gemm_pair_kernel<false>, 2 * s->pair_clusters_dn, kGemmThreads,
                                         kP2SmemBytes, st, dn)
-                             : launch_k(grouped_gemm_kernel<false>, grid, kGemmThreads, kGemmSmemBytes, st, dn)));
+                             : launch_k(grouped_gemm_kernel<false>, grid, kGemmThreadsSm, kGemmSmemBytes, st, dn)));
   }
   if (split) {
     const size_t n4 = static_cast<size_t>(d.T) * d.D / 4;
