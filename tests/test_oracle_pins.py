@@ -134,6 +134,30 @@ def test_top_1_weight_is_one():
     assert np.all(wt == 1.0)
 
 
+def test_skewed_bias_sends_half_the_assignments_to_a_tenth_of_the_experts():
+    """The skewed-routing workload is specified by its effect: a router bias of
+    2 ln(Zipf(1.1) rank probability) per expert, so that 10% of the experts
+    receive more than half of the assignments. Pinned two ways: exp(bias / 2)
+    is the Zipf pmf (sums to one, strictly decreasing with the rank), and on
+    512 seeded tokens routed by the oracle with the benchmark's router weights
+    (the first draw of the weight stream, seed 0) the 13 most-chosen of the
+    128 experts take more than half of the 8 x 512 assignments."""
+    bias = inputs.zipf_router_bias()
+    pmf = np.exp(bias.astype(np.float64) / 2)
+    assert abs(pmf.sum() - 1.0) < 1e-5
+    assert np.all(np.diff(pmf) < 0)
+    w_r = inputs._normal_bf16(inputs._generator(0), (inputs.EMBED_DIM, inputs.NUM_EXPERTS), inputs.INIT_STD)
+    x = inputs.make_x(512)
+    idx, w, _ = mo.route(x, w_r, 8, bias=bias)
+    cnt = np.bincount(idx.ravel(), minlength=inputs.NUM_EXPERTS)
+    assert cnt.sum() == 8 * 512
+    assert np.sort(cnt)[::-1][:13].sum() > 0.5 * cnt.sum()
+    # without the bias the same tokens spread out: no tenth of the experts takes half
+    idx0, _, _ = mo.route(x, w_r, 8)
+    cnt0 = np.bincount(idx0.ravel(), minlength=inputs.NUM_EXPERTS)
+    assert np.sort(cnt0)[::-1][:13].sum() < 0.25 * cnt0.sum()
+
+
 def test_permutation_against_stable_sort():
     """Counting-based permutation == a library stable sort of (expert, token) keys."""
     rng = np.random.default_rng(2)
