@@ -27,6 +27,8 @@
 //   warps 2..9  epilogue, two warps per TMEM lane quarter (each half of the
 //               column chunks): tcgen05.ld the fp32 accumulator, apply GeGLU
 //               or convert, store rows that belong to the tile
+//   warps 10,11 copy warps: lane 0 reads each tile from the ring and issues
+//               copy threads 1 and 2's share of its stages
 // Shared memory: 4 stages x (16 KB A + 32 KB B), 128-byte swizzle.
 // TMEM: 2 accumulator buffers x 256 fp32 columns, so the epilogue of one tile
 // overlaps the main loop of the next.
