@@ -21,7 +21,7 @@ What the block computes, with the passage each step follows:
   GELU); config.json text_config.hidden_activation gelu_pytorch_tanh], widths
   expert_dim = 704 and moe_dense_hidden_dim = 2112 [TransformerConfig].
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * equal logits: the lower expert index ranks first;
 * the order of the k selected experts ("slots") is by descending logit;

@@ -12,7 +12,7 @@ activations are quantised per call ("dynamic": "local") under a scale fixed
 by calibration ("observer": static_minmax). The routers stay bf16 (the
 ``ignore`` list names every ``layers.N.router.proj``).
 
-Reading of the arithmetic the page leaves open (listed in the design doc):
+Reading of the arithmetic the page leaves open:
 
 * tensor scale  G = 448 * 6 / amax(tensor), fp32 (G = 1 for an all-zero tensor);
 * group scale   s = e4m3(fp32(fp32(amax_group / 6) * G)), round to nearest even,

@@ -13,7 +13,7 @@ What it computes, with the passage each step follows:
 * The block's output adds to the residual stream of width embed_dim
   [model card, "Residual stream width": 2816].
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * RMSNorm(v) = gamma * v / sqrt(mean(v^2) + eps), a learned per-channel scale
   gamma [embed_dim] that multiplies (no offset);
