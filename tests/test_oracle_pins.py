@@ -257,11 +257,37 @@ def test_given_routing_reproduces_own_routing():
 
 
 def test_rms_normalize():
+    """Closed forms of x / sqrt(mean(x^2) + 1e-6) (model card: epsilon 1e-06)."""
     rng = np.random.default_rng(0)
-    x = rng.standard_normal((7, 256)) * 3
+    # a constant row c gives c / sqrt(c^2 + eps) everywhere; at c = 1e-3 the
+    # epsilon equals the mean square, so dropping it would give 1, not 1/sqrt(2)
+    for c in (1e-3, -2.0, 3e-4):
+        got = mo.rms_normalize(np.full((1, 96), c))
+        np.testing.assert_allclose(got, c / np.sqrt(c * c + 1e-6), rtol=1e-14)
+    np.testing.assert_allclose(mo.rms_normalize(np.full((1, 8), 1e-3)), 2.0**-0.5, rtol=1e-12)
+    # the output's mean square is ms / (ms + eps) for any row of mean square ms
+    x = rng.standard_normal((7, 256)) * rng.uniform(1e-4, 3, (7, 1))
+    ms = np.mean(x * x, axis=1)
     y = mo.rms_normalize(x)
-    np.testing.assert_allclose(np.mean(y * y, axis=1), 1.0, rtol=1e-5)
-    np.testing.assert_allclose(mo.rms_normalize(5 * x), y, rtol=1e-6)
+    np.testing.assert_allclose(np.mean(y * y, axis=1), ms / (ms + 1e-6), rtol=1e-12)
+    # every row is scaled by one positive factor (direction kept), zero stays zero
+    np.testing.assert_allclose(y / x, (y / x)[:, :1] * np.ones((1, 256)), rtol=1e-12)
+    assert not mo.rms_normalize(np.zeros((2, 16))).any()
+
+
+def test_top_k_gap_brute_force():
+    """k-th minus (k+1)-th largest logit per row, against Python's sorted()."""
+    rng = np.random.default_rng(8)
+    logits = rng.standard_normal((40, 16))
+    logits[3, 5] = logits[3, 9]  # a tie across the k / k+1 boundary
+    logits[3] = np.where(logits[3] > logits[3, 5], -5.0, logits[3])
+    for k in (1, 2, 8, 15):
+        got = mo.top_k_gap(logits, k)
+        for t in range(40):
+            s = sorted(logits[t].tolist(), reverse=True)
+            assert got[t] == s[k - 1] - s[k], (k, t)
+    assert mo.top_k_gap(logits, 1)[3] == 0.0  # the tied pair leads row 3
+    assert np.all(np.isinf(mo.top_k_gap(logits, 16)))
 
 
 # -------------------------------------------------------------------- NVFP4
