@@ -86,6 +86,8 @@ def parse():
     ap.add_argument("--workload", default="decode", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="decode workload: skip the T=4096 prefill run that the default line carries")
     ap.add_argument("--sandwich", action="store_true",
                     help="bf16 workloads: time the block with the pre/post-FFN RMSNorm sandwich and the residual add")
     ap.add_argument("--layers", type=int, default=None, help="nvfp4_stack depth (default 30)")
@@ -285,11 +287,136 @@ def gen_weights_gpu(seed: int = 0, std: float = 0.02):
     )
 
 
+def _bf16_config(wl, T, world, sandwich: bool) -> dict:
+    """The config dict of a bf16 block workload (shared by our arm and the reference arm)."""
+    return {
+        "workload": wl["desc"] + (", with the pre/post-FFN RMSNorm sandwich and residual" if sandwich else ""),
+        "tokens_per_gpu": T,
+        "global_batch": T * world,
+        "parallelism": f"replicas{world}" if world > 1 else "single",
+        "l2": "inputs larger than L2 (1.5 GB of expert weights per step)",
+        "router_bias": "zipf(1.1)" if wl["bias"] else None,
+        "sandwich": bool(sandwich),
+    }
+
+
+def time_block(B, dw, T, bias, steps, warmup, world, local, sandwich, rank=0):
+    """Time one bf16 block workload through the C ABI. Returns a dict with the
+    aggregate, the per-kernel breakdown, the dominant kernel's own timing and
+    the routing statistics.
+
+    Three device-timed passes of `steps` steps each, after `warmup` untimed
+    steps: (1) the headline region, events only at its ends, so every kernel
+    keeps its programmatic-dependent-launch overlap; (2) events around the
+    dominant kernel only (its achieved bandwidth / throughput); the breakdown
+    of every kernel comes from a separate pass with events around each."""
+    import torch
+
+    from mixture_experts_transformer_b200 import block, inputs
+
+    gx = torch.Generator(device="cuda").manual_seed(1 + rank)
+    x = torch.empty((T, D), dtype=torch.float32, device="cuda").normal_(0.0, 1.0, generator=gx).to(torch.bfloat16)
+    out = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    ws, _ = block.workspace_for(inputs.GEMMA4_26B_A4B, T)
+    stream = torch.cuda.current_stream()
+    p = B.make_params(T, x, *dw.args(), out, router_bias=bias, workspace=ws, **sandwich)
+
+    # routing statistics of this batch (outside the timed regions)
+    dbg = block.forward(dw, x, router_bias=bias, debug=True, workspace=ws, **sandwich)
+    torch.cuda.synchronize()
+    cnt = dbg.cnt.cpu().numpy()
+    del dbg
+    st = B.moe_get_device_status()
+    if st != B.MOE_OK:
+        raise RuntimeError(B.moe_status_string(st))
+
+    for _ in range(warmup):
+        B.check(B.moe_block_forward_ex(p, stream), "forward")
+    torch.cuda.synchronize()
+    launches_per_step = B.moe_last_launch_count()
+
+    # per-kernel breakdown: events around every kernel (a pass of its own)
+    B.moe_profile_begin()
+    for _ in range(min(steps, 50)):
+        B.check(B.moe_block_forward_ex(p, stream), "forward")
+    torch.cuda.synchronize()
+    breakdown = B.moe_profile_end()
+    dominant = max(breakdown, key=lambda k: breakdown[k][0])
+
+    # (1) headline: device events around the K steps only
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        e0.record(stream)
+        for _ in range(steps):
+            B.check(B.moe_block_forward_ex(p, stream), "forward")
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = reduce_max(e0.elapsed_time(e1), world)
+
+    # (2) the dominant kernel's own duration, events around it alone
+    torch.cuda.synchronize()
+    B.moe_profile_begin([dominant])
+    for _ in range(steps):
+        B.check(B.moe_block_forward_ex(p, stream), "forward")
+    torch.cuda.synchronize()
+    per_kernel = B.moe_profile_end()
+    st = B.moe_get_device_status()
+    if st != B.MOE_OK:
+        raise RuntimeError(B.moe_status_string(st))
+    return {
+        "x": x, "out": out, "p": p, "ws": ws, "agg": aggregate(T, steps, ms, world), "breakdown": breakdown,
+        "dominant": dominant, "dom_ms": per_kernel[dominant][0] / per_kernel[dominant][1],
+        "clocks": clocks.report(), "cnt": cnt, "touched": int((cnt > 0).sum()),
+        "launches_per_step": launches_per_step,
+    }
+
+
+def roofline_of(res, T, bound, peaks, ms_total) -> tuple[dict, dict]:
+    """(roofline of the dominant kernel, whole-block roofline) for a bf16 block run."""
+    dominant, dom_ms, touched, cnt = res["dominant"], res["dom_ms"], res["touched"], res["cnt"]
+    byts, flops = algorithmic(dominant, T, touched, cnt)
+    long_region = ms_total / 1e3 > 2.0
+    if bound == "hbm":
+        achieved = byts / (dom_ms / 1e3) / 1e9
+        peak, unit, peak_name = peaks["hbm_gbs"], "GB/s", "hbm_gbs"
+    else:
+        achieved = flops / (dom_ms / 1e3) / 1e12
+        peak_name = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        peak, unit = peaks[peak_name], "TFLOP/s"
+    step_ms = res["agg"]["ms_per_step"]
+    weight_bytes = touched * BYTES_PER_EXPERT + SHARED_BYTES + ROUTER_BYTES
+    roof = {
+        "bound": bound,
+        "kernel": dominant,
+        "achieved": achieved,
+        "peak": peak,
+        "peak_source": f"{peaks['source']} {peak_name}",
+        "unit": unit,
+        "frac": achieved / peak,
+        "traffic": None,
+        "algorithmic_bytes": byts,
+        "algorithmic_flops": flops,
+        "kernel_ms": dom_ms,
+        "kernel_timing": "a pass of its own of the same steps, events around this kernel only",
+    }
+    block_roof = {
+        "hbm_touched_weights_gbs": weight_bytes / (step_ms / 1e3) / 1e9,
+        "hbm_frac": weight_bytes / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "tensor_tflops": T * FLOP_PER_TOKEN_GEMM / (step_ms / 1e3) / 1e12,
+        "tensor_frac": T * FLOP_PER_TOKEN_GEMM / (step_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "touched_experts": touched,
+    }
+    return roof, block_roof
+
+
 def run_ours(args, world, rank, local):
     import torch
 
     from mixture_experts_transformer_b200 import binding as B
-    from mixture_experts_transformer_b200 import block, build, inputs
+    from mixture_experts_transformer_b200 import build, inputs
 
     if rank == 0:
         build.build()
@@ -299,12 +426,7 @@ def run_ours(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     T = wl["T"]
     dw = gen_weights_gpu(seed=0)
-    gx = torch.Generator(device="cuda").manual_seed(1 + rank)
-    x = torch.empty((T, D), dtype=torch.float32, device="cuda").normal_(0.0, 1.0, generator=gx).to(torch.bfloat16)
     bias = torch.from_numpy(inputs.zipf_router_bias()).cuda() if wl["bias"] else None
-    out = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
-    ws, _ = block.workspace_for(inputs.GEMMA4_26B_A4B, T)
-    stream = torch.cuda.current_stream()
     sandwich = {}
     if args.sandwich:
         # learned scales of the pre- and post-FFN RMSNorm, seeded U(0.5, 1.5)
@@ -314,50 +436,10 @@ def run_ours(args, world, rank, local):
             "norm_post": torch.empty(D, device="cuda").uniform_(0.5, 1.5, generator=gs).to(torch.bfloat16),
             "residual": True,
         }
-    p = B.make_params(T, x, *dw.args(), out, router_bias=bias, workspace=ws, **sandwich)
-
-    # routing statistics of this batch (outside the timed region)
-    dbg = block.forward(dw, x, router_bias=bias, debug=True, workspace=ws, **sandwich)
-    torch.cuda.synchronize()
-    cnt = dbg.cnt.cpu().numpy()
-    touched = int((cnt > 0).sum())
-    st = B.moe_get_device_status()
-    if st != B.MOE_OK:
-        raise RuntimeError(B.moe_status_string(st))
-
-    for _ in range(args.warmup):
-        B.check(B.moe_block_forward_ex(p, stream), "forward")
-    torch.cuda.synchronize()
-    launches_per_step = B.moe_last_launch_count()
-
-    # ---- per-kernel breakdown: events around every kernel (untimed pass)
-    B.moe_profile_begin()
-    for _ in range(min(args.steps, 50)):
-        B.check(B.moe_block_forward_ex(p, stream), "forward")
-    torch.cuda.synchronize()
-    breakdown = B.moe_profile_end()
-    dominant = max(breakdown, key=lambda k: breakdown[k][0])
-
-    # ---- timed region: device events around the K steps; events around the
-    # dominant kernel only, so the other kernels keep their launch overlap
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        B.moe_profile_begin([dominant])
-        e0.record(stream)
-        for _ in range(args.steps):
-            B.check(B.moe_block_forward_ex(p, stream), "forward")
-        e1.record(stream)
-        torch.cuda.synchronize()
-        per_kernel = B.moe_profile_end()
-    barrier(world)
-    ms_local = e0.elapsed_time(e1)
-    ms = reduce_max(ms_local, world)
-    agg = aggregate(T, args.steps, ms, world)
-    st = B.moe_get_device_status()
-    if st != B.MOE_OK:
-        raise RuntimeError(B.moe_status_string(st))
+    res_t = time_block(B, dw, T, bias, args.steps, args.warmup, world, local, sandwich, rank)
+    x, out, p = res_t["x"], res_t["out"], res_t["p"]
+    agg = res_t["agg"]
+    stream = torch.cuda.current_stream()
 
     # ---- end to end: host buffers through the C ABI, copies inside the timed region
     x_host = x.cpu().pin_memory()
@@ -378,32 +460,25 @@ def run_ours(args, world, rank, local):
     barrier(world)
     if not torch.equal(out_host, out.cpu()):
         raise RuntimeError("host-buffer path disagrees with the device path")
+    ws_bytes = res_t["ws"].numel()
+    del res_t["ws"], res_t["x"], res_t["out"], res_t["p"]
+
+    # ---- the metric's prefill half: the T = 4096 block, timed the same way
+    prefill = None
+    if args.workload == "decode" and not args.no_prefill:
+        wp = WORKLOADS["prefill"]
+        torch.cuda.empty_cache()
+        res_p = time_block(B, dw, wp["T"], None, args.steps, args.warmup, world, local, sandwich, rank)
+        del res_p["ws"], res_p["x"], res_p["out"], res_p["p"]
+        prefill = res_p
 
     if rank != 0:
         return None
 
     peaks = measured_peaks()
-    kernel_ms = {k: v[0] / v[1] for k, v in breakdown.items()}
-    byts, flops = algorithmic(dominant, T, touched, cnt)
-    dom_ms = per_kernel[dominant][0] / per_kernel[dominant][1]
-    long_region = ms / 1e3 > 2.0
-    if wl["bound"] == "hbm":
-        achieved = byts / (dom_ms / 1e3) / 1e9
-        peak, unit, peak_name = peaks["hbm_gbs"], "GB/s", "hbm_gbs"
-    else:
-        achieved = flops / (dom_ms / 1e3) / 1e12
-        key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
-        peak, unit, peak_name = peaks[key], "TFLOP/s", key
-    traffic = ncu_traffic(dominant, args.workload)
     step_ms = agg["ms_per_step"]
-    weight_bytes = touched * BYTES_PER_EXPERT + SHARED_BYTES + ROUTER_BYTES
-    block_roof = {
-        "hbm_touched_weights_gbs": weight_bytes / (step_ms / 1e3) / 1e9,
-        "hbm_frac": weight_bytes / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-        "tensor_tflops": T * FLOP_PER_TOKEN_GEMM / (step_ms / 1e3) / 1e12,
-        "tensor_frac": T * FLOP_PER_TOKEN_GEMM / (step_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
-        "touched_experts": touched,
-    }
+    roof, block_roof = roofline_of(res_t, T, wl["bound"], peaks, agg["ms_per_step"] * args.steps)
+    roof["traffic"] = ncu_traffic(res_t["dominant"], args.workload)
     res = {
         "metric": METRIC,
         "value": agg["value"],
@@ -417,39 +492,38 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, x ~ N(0,1)",
-        "config": {
-            "workload": wl["desc"] + (", with the pre/post-FFN RMSNorm sandwich and residual" if args.sandwich else ""),
-            "tokens_per_gpu": T,
-            "global_batch": T * world,
-            "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": "inputs larger than L2 (1.5 GB of expert weights per step)",
-            "router_bias": "zipf(1.1)" if wl["bias"] else None,
-            "sandwich": bool(args.sandwich),
-        },
-        "roofline": {
-            "bound": wl["bound"],
-            "kernel": dominant,
-            "achieved": achieved,
-            "peak": peak,
-            "peak_source": f"{peaks['source']} {peak_name}",
-            "unit": unit,
-            "frac": achieved / peak,
-            "traffic": traffic,
-            "algorithmic_bytes": byts,
-            "algorithmic_flops": flops,
-            "kernel_ms": dom_ms,
-        },
+        "config": _bf16_config(wl, T, world, args.sandwich),
+        "roofline": roof,
         "block_roofline": block_roof,
-        "kernels_ms_per_launch": kernel_ms,
-        "gpu_launches": launches_per_step * args.steps,
+        "kernels_ms_per_launch": {k: v[0] / v[1] for k, v in res_t["breakdown"].items()},
+        "gpu_launches": res_t["launches_per_step"] * args.steps,
         "e2e": {
             "value": T * args.steps * world / (e2e_ms / 1e3),
             "unit": "tokens/s",
             "h2d_bytes_per_step": T * D * 2,
             "d2h_bytes_per_step": T * D * 2,
         },
-        "clocks": clocks.report(),
+        "clocks": res_t["clocks"],
+        "workspace_bytes": ws_bytes,
     }
+    if prefill is not None:
+        wp = WORKLOADS["prefill"]
+        proof, pblock = roofline_of(prefill, wp["T"], wp["bound"], peaks, prefill["agg"]["ms_per_step"] * args.steps)
+        proof["traffic"] = ncu_traffic(prefill["dominant"], "prefill")
+        res["prefill"] = {
+            "metric": METRIC,
+            "value": prefill["agg"]["value"],
+            "unit": "tokens/s",
+            "ms_per_step": prefill["agg"]["ms_per_step"],
+            "steps": args.steps,
+            "config": _bf16_config(wp, wp["T"], world, args.sandwich),
+            "roofline": proof,
+            "block_roofline": pblock,
+            "tensor_frac": pblock["tensor_frac"],
+            "kernels_ms_per_launch": {k: v[0] / v[1] for k, v in prefill["breakdown"].items()},
+            "gpu_launches": prefill["launches_per_step"] * args.steps,
+            "clocks": prefill["clocks"],
+        }
     if world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(dw, x, bias, T, budget_s=12.0, sandwich=sandwich)
     return res
@@ -717,7 +791,15 @@ def run_reference(args, world, rank):
 
     wl = WORKLOADS[args.workload]
     T = wl["T"]
-    n = min(T, 8)
+    if args.workload == "nvfp4_stack":
+        # one oracle step re-quantises the weights of every touched expert
+        # (~126 x 3 matrices per layer, minutes per layer on the host)
+        return {"impl": "reference", "unavailable": "the oracle's NVFP4 block needs minutes of host time per layer "
+                "(it re-quantises every touched expert's weights per call), beyond a bounded step; this workload's "
+                "own line carries its cpu_baseline (one token through the first layers, scaled)"}
+    # the same bounded sample as our arm's cpu_baseline leg: the first 64
+    # tokens of the batch (the whole batch at the decode workload)
+    n = min(T, 64)
     metric = METRIC
     if wl.get("dense"):
         dw = inputs.make_dense_weights()
@@ -761,21 +843,26 @@ def run_reference(args, world, rank):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, x ~ N(0,1)",
-        "config": {
-            "workload": wl["desc"] + (", with the pre/post-FFN RMSNorm sandwich and residual" if args.sandwich else ""),
-            "tokens_per_gpu": T,
-            "global_batch": T * world,
-            "parallelism": "single",
-            "sandwich": bool(args.sandwich),
-        },
+        "config": _dense_config(wl, T, world) if wl.get("dense") else _bf16_config(wl, T, world, args.sandwich),
         "cpu_baseline": {
             "value": v,
             "unit": "tokens/s",
             "cores": cores,
             "kind": "oracle",
-            "sample": f"each step: the first {n} of the workload's {T} tokens through the fp64 oracle",
+            "sample": f"each step: the first {n} of the workload's {T} tokens through the fp64 oracle"
+            + ("" if n == T else f", scaled to tokens/s per token (tokens are independent in the block)"),
         },
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def _dense_config(wl, T, world) -> dict:
+    return {
+        "workload": wl["desc"],
+        "tokens_per_gpu": T,
+        "global_batch": T * world,
+        "parallelism": f"replicas{world}" if world > 1 else "single",
+        "l2": "weights 157 MB, larger than L2",
     }
 
 
@@ -884,13 +971,7 @@ def run_dense(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic: seeded N(0,0.02) random-init weights of the published E4B FFN shapes, x ~ N(0,1)",
-        "config": {
-            "workload": wl["desc"],
-            "tokens_per_gpu": T,
-            "global_batch": T * world,
-            "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": "weights 157 MB, larger than L2",
-        },
+        "config": _dense_config(wl, T, world),
         "roofline": {
             "bound": wl["bound"],
             "kernel": dominant,

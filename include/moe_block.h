@@ -90,7 +90,10 @@ typedef enum {
  *     them one after another or give each its own workspace);
  *   out_f32 [T, embed_dim] fp32: the pre-rounding output (out == RNE(out_f32));
  *   idx_out [T, top_k] int32, w_out [T, top_k] fp32: the routing used;
- *   cnt_out [num_experts] int32: tokens per expert.
+ *   cnt_out [num_experts] int32: tokens per expert;
+ *   logits_out [T, num_experts] fp32: the router logits the selection used
+ *     (router_bias included), a debug output (also honoured by moe_route and
+ *     moe_route_noalloc).
  *
  * The normalisation sandwich around the block (model card: RMSNorm layers,
  * "sandwich" = pre and post, epsilon 1e-06), each part optional:
@@ -102,6 +105,23 @@ typedef enum {
  *   residual  nonzero: out = RNE(x + that), the raw input x added in fp32.
  * With any of the three, embed_dim must be <= 4096 (a row per CTA). out_f32
  * then holds the final pre-rounding value.
+ *
+ * Expert parallelism (the layer split over G devices, each holding 1/G of the
+ * experts and a 1/G slice of the shared MLP's hidden units): an expert shard
+ * owns experts [expert_begin, expert_begin + expert_count) of the
+ * num_experts the router scores (expert_count 0 = all of them). Then wg, wu,
+ * wd hold only those experts ([expert_count, ...], expert 0 of the arrays
+ * being expert_begin); w_router still covers every expert, so routing and
+ * weights are those of the whole layer; sg, su, sd are the shard's slice of
+ * the shared MLP (hidden_dim = the slice width, sg / su its columns, sd its
+ * rows). The call then computes the shard's partial sum
+ *   s_slice[t] + sum over the slots j whose expert is local of w[t, j] y_j[t],
+ * slots in order, in fp32; the partial sums of all shards add up to the
+ * block's output (GeGLU acts per hidden unit, so the shared MLP splits
+ * exactly over its hidden units). The caller sums them across devices (e.g.
+ * a reduce-scatter) and rounds with moe_round_bf16. A shard may not use
+ * norm_post or residual, which act on the full sum.
+ * out may be NULL when out_f32 is given: only the fp32 result is written.
  */
 typedef struct moe_params {
   int T;
@@ -129,6 +149,9 @@ typedef struct moe_params {
   const void* norm_pre;
   const void* norm_post;
   int residual;
+  float* logits_out;
+  int expert_begin;
+  int expert_count;
 } moe_params;
 
 /*
@@ -236,14 +259,15 @@ const char* moe_kernel_name(int id);
  * reserved up front, which forbid libraries to call cudaMalloc behind their
  * back, and runtimes whose allocation calls would stall or fail mid-run).
  *
- * Same arguments, kernels and results as moe_route (idx and w are caller
- * memory; the workspace fields of p are ignored). Its scratch - the split-K
- * partial logits and the token-expert bitmasks - lives in a fixed 4 MiB
- * __device__ array inside the library, which every GPU that loads the library
- * holds until the process exits. T is limited to 4096 tokens (and the scratch
- * must fit: the split of the reduction is narrowed when needed); a larger
- * batch returns MOE_ERR_WORKSPACE before anything is enqueued. No cudaMalloc,
- * cudaFree or allocating library routine is called.
+ * Same arguments, kernels, split of the reduction and therefore bit-identical
+ * results as moe_route (idx, w and the optional logits_out are caller memory;
+ * the workspace fields of p are ignored). Its scratch - the split-K partial
+ * logits and the token-expert bitmasks - lives in a fixed 10 MiB __device__
+ * array inside the library, which every GPU that loads the library holds until
+ * the process exits; that size holds moe_route's own split at every batch up
+ * to the limit. T is limited to 4096 tokens; a larger batch returns
+ * MOE_ERR_WORKSPACE before anything is enqueued. No cudaMalloc, cudaFree or
+ * allocating library routine is called.
  *
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) once for that device; make that first call before
@@ -335,16 +359,45 @@ typedef struct moe_nvfp4_params {
 
 size_t moe_nvfp4_workspace_bytes(const moe_nvfp4_params* p);
 
+/*
+ * Where the NVFP4 block's intermediates live inside its workspace (byte
+ * offsets). Routed rows are padded per expert to whole 128-row blocks
+ * (routed_rows rows in all); token-order buffers have token_rows rows (T
+ * rounded up to 128). Codes are e2m1 [rows][K/2] (element 2j in the low
+ * nibble of byte j), group scales e4m3 in 512-byte atoms [rows/128][K/64][512]
+ * (row r, 16-group c of the 64-K block at byte 16*(r%32) + 4*(r/32%4) + c):
+ *   xq_perm / xsf_perm  x quantised, routed-row order (K = embed_dim)
+ *   xq_tok / xsf_tok    x quantised, token order
+ *   hq / hsf            routed GeGLU rows quantised under g_h (K = expert_dim)
+ *   hsq / hssf          shared GeGLU rows quantised under g_hs (K = hidden_dim)
+ *   y [routed_rows, embed_dim] bf16, s [T, embed_dim] fp32
+ *   idx, w, cnt, off, row_of as in moe_ws_layout (row_of: the padded routed row)
+ */
+typedef struct moe_nvfp4_ws_layout {
+  size_t total_bytes;
+  size_t xq_perm, xsf_perm, xq_tok, xsf_tok;
+  size_t hq, hsf, hsq, hssf;
+  size_t y, s;
+  size_t idx, w, cnt, off, row_of;
+  long long routed_rows, token_rows;
+} moe_nvfp4_ws_layout;
+
+moe_status moe_nvfp4_workspace_layout(const moe_nvfp4_params* p, moe_nvfp4_ws_layout* out);
+
 /* One NVFP4 block forward pass (router bf16, expert and shared Linears NVFP4). */
 moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream);
 
 /*
- * Calibration observer for the NVFP4 activation scales: runs the bf16 block on
- * p (which must carry a caller workspace) and writes amax[0] = max |x|,
- * amax[1] = max |h| over the routed GeGLU rows, amax[2] = max |hs| over the
- * shared GeGLU rows (device fp32 [3]). The tensor scales are 448*6/amax.
+ * Calibration observer for the NVFP4 activation scales (the checkpoint's
+ * input_activations observer static_minmax): runs the bf16 block on p (which
+ * must carry a caller workspace) and writes, in device fp32 [3] buffers,
+ * amax[0] = max |x| (the block input, after norm_pre when given), amax[1] =
+ * max |h| over the routed GeGLU rows, amax[2] = max |hs| over the shared
+ * GeGLU rows, and the tensor scales scales[i] = RN(448 * 6 / amax[i]) (1 for
+ * an all-zero tensor): g_x, g_h, g_hs of moe_nvfp4_params. amax and scales
+ * must not overlap. The GeGLU rows are observed as stored, in bf16.
  */
-moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream);
+moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, float* scales, void* stream);
 
 /* -------------------------------------------------------- dense GeGLU FFN
  *
@@ -381,6 +434,13 @@ typedef struct moe_dense_params {
 
 size_t moe_dense_workspace_bytes(const moe_dense_params* p);
 moe_status moe_dense_ffn_forward(const moe_dense_params* p, void* stream);
+
+/*
+ * out[i] = RNE_bf16(in[i]) for i < n (fp32 in, bf16 out; n a multiple of 8,
+ * both 16-byte aligned, not overlapping): the final rounding of an output
+ * summed across expert shards.
+ */
+moe_status moe_round_bf16(const float* in, void* out, size_t n, void* stream);
 
 /* Human-readable name of a status code. */
 const char* moe_status_string(moe_status s);

@@ -53,6 +53,9 @@ class MoeParams(ctypes.Structure):
         ("norm_pre", _vp),
         ("norm_post", _vp),
         ("residual", ctypes.c_int),
+        ("logits_out", _vp),
+        ("expert_begin", ctypes.c_int),
+        ("expert_count", ctypes.c_int),
     ]
 
 
@@ -76,6 +79,7 @@ EXPORTS = {
     "moe_debug_timeout_probe": (ctypes.c_int, [ctypes.c_int, _vp]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_launch_count": (ctypes.c_int, []),
+    "moe_round_bf16": (ctypes.c_int, [_vp, _vp, ctypes.c_size_t, _vp]),
     "moe_block_forward_hostio": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp, _vp]),
     "moe_profile_begin": (ctypes.c_int, [ctypes.c_uint32]),
     "moe_profile_end": (ctypes.c_int, [_vp, _vp, ctypes.c_int]),
@@ -157,6 +161,9 @@ def make_params(
     norm_pre=None,
     norm_post=None,
     residual: bool = False,
+    logits_out=None,
+    expert_begin: int = 0,
+    expert_count: int = 0,
 ) -> MoeParams:
     p = MoeParams()
     p.T = T
@@ -186,9 +193,11 @@ def make_params(
         ("workspace", workspace),
         ("norm_pre", norm_pre),
         ("norm_post", norm_post),
+        ("logits_out", logits_out),
     ):
         setattr(p, name, ptr(val))
     p.residual = 1 if residual else 0
+    p.expert_begin, p.expert_count = expert_begin, expert_count
     if workspace is not None and not workspace_bytes:
         workspace_bytes = workspace.numel() * workspace.element_size()
     p.workspace_bytes = workspace_bytes
@@ -243,6 +252,10 @@ def moe_status_string(status: int) -> str:
 
 def moe_last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+def moe_round_bf16(src, dst, n: int, stream=None) -> int:
+    return lib().moe_round_bf16(ptr(src), ptr(dst), n, stream_handle(stream))
 
 
 def moe_block_forward_hostio(p: MoeParams, x_host, out_host, stream=None) -> int:
@@ -327,6 +340,14 @@ class MoeNvfp4Params(ctypes.Structure):
     ]
 
 
+class MoeNvfp4WsLayout(ctypes.Structure):
+    _fields_ = [
+        (name, ctypes.c_size_t)
+        for name in ("total_bytes", "xq_perm", "xsf_perm", "xq_tok", "xsf_tok", "hq", "hsf", "hsq", "hssf", "y", "s",
+                     "idx", "w", "cnt", "off", "row_of")
+    ] + [("routed_rows", ctypes.c_longlong), ("token_rows", ctypes.c_longlong)]
+
+
 EXPORTS.update(
     {
         "moe_nvfp4_weight_bytes": (
@@ -339,8 +360,10 @@ EXPORTS.update(
         ),
         "moe_nvfp4_quantize_act": (ctypes.c_int, [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_float, _vp, _vp, _vp]),
         "moe_nvfp4_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeNvfp4Params)]),
+        "moe_nvfp4_workspace_layout": (ctypes.c_int, [ctypes.POINTER(MoeNvfp4Params),
+                                                      ctypes.POINTER(MoeNvfp4WsLayout)]),
         "moe_block_forward_nvfp4": (ctypes.c_int, [ctypes.POINTER(MoeNvfp4Params), _vp]),
-        "moe_nvfp4_calibrate": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp]),
+        "moe_nvfp4_calibrate": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp, _vp]),
     }
 )
 
@@ -363,12 +386,18 @@ def moe_nvfp4_workspace_bytes(p: MoeNvfp4Params) -> int:
     return lib().moe_nvfp4_workspace_bytes(ctypes.byref(p))
 
 
+def moe_nvfp4_workspace_layout(p: MoeNvfp4Params) -> "MoeNvfp4WsLayout":
+    out = MoeNvfp4WsLayout()
+    check(lib().moe_nvfp4_workspace_layout(ctypes.byref(p), ctypes.byref(out)), "moe_nvfp4_workspace_layout")
+    return out
+
+
 def moe_block_forward_nvfp4(p: MoeNvfp4Params, stream=None) -> int:
     return lib().moe_block_forward_nvfp4(ctypes.byref(p), stream_handle(stream))
 
 
-def moe_nvfp4_calibrate(p: MoeParams, amax, stream=None) -> int:
-    return lib().moe_nvfp4_calibrate(ctypes.byref(p), ptr(amax), stream_handle(stream))
+def moe_nvfp4_calibrate(p: MoeParams, amax, scales, stream=None) -> int:
+    return lib().moe_nvfp4_calibrate(ctypes.byref(p), ptr(amax), ptr(scales), stream_handle(stream))
 
 
 # ------------------------------------------------------------ dense GeGLU FFN

@@ -48,6 +48,7 @@ class BlockResult:
     idx: torch.Tensor | None = None
     w: torch.Tensor | None = None
     cnt: torch.Tensor | None = None
+    logits: torch.Tensor | None = None
 
 
 def forward(
@@ -64,7 +65,7 @@ def forward(
     norm_post: torch.Tensor | None = None,
     residual: bool = False,
 ) -> BlockResult:
-    """Run one block; with debug=True also return out_f32, the routing and the counts.
+    """Run one block; with debug=True also return out_f32, the routing, the router logits and the counts.
     norm_pre / norm_post (bf16 [embed_dim]) and residual add the normalisation
     sandwich: out = x + norm_post-RMSNorm(block(norm_pre-RMSNorm(x)))."""
     T = x.shape[0]
@@ -77,6 +78,7 @@ def forward(
         res.idx = torch.empty((T, top_k), dtype=torch.int32, device=dev)
         res.w = torch.empty((T, top_k), dtype=torch.float32, device=dev)
         res.cnt = torch.empty((dw.dims.num_experts,), dtype=torch.int32, device=dev)
+        res.logits = torch.empty((T, dw.dims.num_experts), dtype=torch.float32, device=dev)
     p = B.make_params(
         T,
         x,
@@ -93,6 +95,7 @@ def forward(
         norm_pre=norm_pre,
         norm_post=norm_post,
         residual=residual,
+        logits_out=res.logits,
     )
     B.check(B.moe_block_forward_ex(p, stream), "moe_block_forward_ex")
     return res
@@ -205,15 +208,18 @@ def nvfp4_params(nw, T, x, out, act_scales, *, top_k=B.TOP_K, router_bias=None, 
 
 
 def calibrate(dw: DeviceWeights, x: torch.Tensor, top_k: int = B.TOP_K, router_bias=None, stream=None):
-    """Static NVFP4 activation tensor scales (g_x, g_h, g_hs) = 448*6/amax from one
-    calibration batch run through the bf16 block (the library's observer)."""
+    """Static NVFP4 activation tensor scales (g_x, g_h, g_hs) from one calibration
+    batch run through the bf16 block: the library's observer writes the amax
+    values and the scales on the device; they are copied back here.
+    Returns ((g_x, g_h, g_hs) as float32, amax [3] float32)."""
     ws, _ = workspace_for(dw.dims, x.shape[0], top_k, device=x.device)
     out = torch.empty((x.shape[0], dw.dims.embed_dim), dtype=torch.bfloat16, device=x.device)
     amax = torch.zeros(3, dtype=torch.float32, device=x.device)
+    scales = torch.zeros(3, dtype=torch.float32, device=x.device)
     p = B.make_params(x.shape[0], x, *dw.args(), out, top_k=top_k, dims=dw.dims, router_bias=router_bias, workspace=ws)
-    B.check(B.moe_nvfp4_calibrate(p, amax, stream), "moe_nvfp4_calibrate")
-    a = amax.cpu().numpy().astype(np.float32)
-    return tuple(np.float32(2688.0) / v if v > 0 else np.float32(1.0) for v in a), a
+    B.check(B.moe_nvfp4_calibrate(p, amax, scales, stream), "moe_nvfp4_calibrate")
+    g = scales.cpu().numpy().astype(np.float32)
+    return tuple(np.float32(v) for v in g), amax.cpu().numpy().astype(np.float32)
 
 
 # ---------------------------------------------------------------- dense FFN

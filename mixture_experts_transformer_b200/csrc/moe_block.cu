@@ -33,6 +33,7 @@ thread_local int t_launches = 0;
 
 struct Dims {
   int T, k, D, E, F, S;
+  int e0 = 0, el = 0;  // expert shard: experts [e0, e0 + el) of the E the router scores (el = E: all)
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -113,10 +114,13 @@ Dims dims_of(const moe_params* p) {
   d.E = p->num_experts ? p->num_experts : MOE_NUM_EXPERTS;
   d.F = p->expert_dim ? p->expert_dim : MOE_EXPERT_DIM;
   d.S = p->hidden_dim ? p->hidden_dim : MOE_HIDDEN_DIM;
+  d.e0 = p->expert_begin;
+  d.el = p->expert_count ? p->expert_count : d.E - d.e0;
   return d;
 }
 
 bool dims_ok(const Dims& d) {
+  if (d.e0 < 0 || d.el < 1 || d.e0 > d.E - d.el) return false;
   if (d.T < 0) return false;
   if (d.D <= 0 || d.F <= 0 || d.S <= 0 || d.D % 64 || d.F % 64 || d.S % 64) return false;
   if (d.E < 8 || d.E > 128 || d.E % 8) return false;
@@ -394,18 +398,22 @@ moe_status check_block_args(const moe_params* p, Dims* d) {
   *d = dims_of(p);
   if (!dims_ok(*d)) return MOE_ERR_INVALID_ARG;
   if (d->T == 0) return MOE_OK;
-  const void* req[] = {p->x, p->w_router, p->wg, p->wu, p->wd, p->sg, p->su, p->sd, p->out};
+  const void* req[] = {p->x, p->w_router, p->wg, p->wu, p->wd, p->sg, p->su, p->sd};
   for (const void* q : req)
     if (!q) return MOE_ERR_INVALID_ARG;
   for (const void* q : req)
     if (!aligned16(q)) return MOE_ERR_ALIGNMENT;
-  if (p->out_f32 && !aligned16(p->out_f32)) return MOE_ERR_ALIGNMENT;
-  const void* opt4[] = {p->router_bias, p->idx_out, p->w_out, p->cnt_out};
+  if (!p->out && !p->out_f32) return MOE_ERR_INVALID_ARG;  // an output is needed
+  if ((p->out && !aligned16(p->out)) || (p->out_f32 && !aligned16(p->out_f32))) return MOE_ERR_ALIGNMENT;
+  // a shard's output is a partial sum: the post-norm and residual act on the full sum
+  if (d->el != d->E && (p->norm_post || p->residual)) return MOE_ERR_INVALID_ARG;
+  if (!p->out && (p->norm_post || p->residual)) return MOE_ERR_INVALID_ARG;
+  const void* opt4[] = {p->router_bias, p->idx_out, p->w_out, p->cnt_out, p->logits_out};
   for (const void* q : opt4)
     if (q && !aligned4(q)) return MOE_ERR_ALIGNMENT;
   const uintptr_t xb = reinterpret_cast<uintptr_t>(p->x), ob = reinterpret_cast<uintptr_t>(p->out);
   const uintptr_t bytes = static_cast<uintptr_t>(d->T) * d->D * 2;
-  if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
+  if (p->out && xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
   if ((p->norm_pre && !aligned16(p->norm_pre)) || (p->norm_post && !aligned16(p->norm_post))) return MOE_ERR_ALIGNMENT;
   if ((p->norm_pre || p->norm_post || p->residual) && d->D > kCombThreads * kCombVec * 8) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
@@ -427,7 +435,7 @@ moe_status resolve_workspace(const moe_params* p, DeviceState* s, const Layout& 
 // ---------------------------------------------------------------- stages
 
 moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void* x, const void* wr,
-                         const float* bias, int32_t* idx, float* w, cudaStream_t st) {
+                         const float* bias, int32_t* idx, float* w, cudaStream_t st, float* logits_out = nullptr) {
   float* partial = reinterpret_cast<float*>(ws + L.partial);
   uint32_t* masks = reinterpret_cast<uint32_t*>(ws + L.masks);
   DeviceState* s = nullptr;
@@ -451,9 +459,9 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
   const int tk_blocks = (d.T + kTopkWarps - 1) / kTopkWarps;
   const cudaError_t le_ =
       L.nsplit > 8 ? launch_k(router_topk_kernel<true>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
-                              L.nsplit, d.k, idx, w, masks)
+                              L.nsplit, d.k, idx, w, masks, logits_out)
                    : launch_k(router_topk_kernel<false>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
-                              L.nsplit, d.k, idx, w, masks);
+                              L.nsplit, d.k, idx, w, masks, logits_out);
   return ls_.done(le_);
 }
 
@@ -471,7 +479,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
                                      reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256,
-                                     paired_gateup(d) ? 1 : 0, (pairs || paired_down(d)) ? 1 : 0);
+                                     paired_gateup(d) ? 1 : 0, (pairs || paired_down(d)) ? 1 : 0, d.e0, d.el);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
@@ -479,7 +487,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
   LaunchScope ls_(kKRouteScatter, st);
   const cudaError_t le_ = launch_k(route_scatter_kernel, blocks, 256, 0, st, idx, masks, base, d.T, d.k, d.E, d.D,
                                    static_cast<const __nv_bfloat16*>(x), row_of, token_of,
-                                   reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm), R, s->err);
+                                   reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm), R, s->err, d.e0, d.el);
   return ls_.done(le_);
 }
 
@@ -509,24 +517,24 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
                               static_cast<const __nv_bfloat16*>(p->norm_pre), d.T, d.D, xn)));
     xin = xn;
   }
-  MOE_TRY(enqueue_route(d, L, ws, xin, p->w_router, p->router_bias, idx, w, st));
+  MOE_TRY(enqueue_route(d, L, ws, xin, p->w_router, p->router_bias, idx, w, st, p->logits_out));
   MOE_TRY(enqueue_permute(d, L, ws, idx, xin, cnt, off, row_of, token_of, st));
 
   // gate|up: experts (problem 0) and shared MLP (problem 1)
   GemmParams gu;
   std::memset(&gu, 0, sizeof(gu));
-  bool ok = map_2d(&gu.tmA[0], x_perm, R, d.D, kBM) && map_3d(&gu.tmB0[0], p->wg, d.E, d.D, d.F) &&
-            map_3d(&gu.tmB1[0], p->wu, d.E, d.D, d.F) && map_2d(&gu.tmA[1], xin, d.T, d.D, kBM) &&
+  bool ok = map_2d(&gu.tmA[0], x_perm, R, d.D, kBM) && map_3d(&gu.tmB0[0], p->wg, d.el, d.D, d.F) &&
+            map_3d(&gu.tmB1[0], p->wu, d.el, d.D, d.F) && map_2d(&gu.tmA[1], xin, d.T, d.D, kBM) &&
             map_3d(&gu.tmB0[1], p->sg, 1, d.D, d.S) && map_3d(&gu.tmB1[1], p->su, 1, d.D, d.S);
   if (!ok) return MOE_ERR_CUDA;
-  gu.prob[0] = GemmProblem{d.D, d.F, d.E, static_cast<int>(R), h, d.F, 0};
+  gu.prob[0] = GemmProblem{d.D, d.F, d.el, static_cast<int>(R), h, d.F, 0};
   gu.prob[1] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
   gu.nprob = 2;
   gu.stream_weights = stream_weights(d) ? 1 : 0;
   gu.a_wide = paired_gateup(d) ? 1 : 0;
   gu.a_small = paired_gateup(d) ? 0 : 1;
   gu.bw_chunks = 2;  // 128 output columns of each projection
-  set_wide_maps(&gu, 0, x_perm, R, d.D, gu.a_wide, p->wg, p->wu, d.E, d.F, 2);
+  set_wide_maps(&gu, 0, x_perm, R, d.D, gu.a_wide, p->wg, p->wu, d.el, d.F, 2);
   set_wide_maps(&gu, 1, xin, d.T, d.D, gu.a_wide, p->sg, p->su, 1, d.S, 2);
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
@@ -544,12 +552,12 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   // down: experts -> y (bf16), shared -> s (fp32)
   GemmParams dn;
   std::memset(&dn, 0, sizeof(dn));
-  ok = map_2d(&dn.tmA[0], h, R, d.F, kBM) && map_3d(&dn.tmB0[0], p->wd, d.E, d.F, d.D) &&
+  ok = map_2d(&dn.tmA[0], h, R, d.F, kBM) && map_3d(&dn.tmB0[0], p->wd, d.el, d.F, d.D) &&
        map_2d(&dn.tmA[1], hs, d.T, d.S, kBM) && map_3d(&dn.tmB0[1], p->sd, 1, d.S, d.D);
   if (!ok) return MOE_ERR_CUDA;
   dn.tmB1[0] = dn.tmB0[0];
   dn.tmB1[1] = dn.tmB0[1];
-  dn.prob[0] = GemmProblem{d.F, d.D, d.E, static_cast<int>(R), y, d.D, 0};
+  dn.prob[0] = GemmProblem{d.F, d.D, d.el, static_cast<int>(R), y, d.D, 0};
   dn.prob[1] = GemmProblem{d.S, d.D, 1, d.T, sbuf, d.D, 1};
   dn.nprob = 2;
   dn.stream_weights = gu.stream_weights;
@@ -557,7 +565,7 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   dn.bw_chunks = pair_sm(d, s) ? 2 : 4;
   dn.a_wide = paired_down(d) && !pair_sm(d, s) ? 1 : 0;
   dn.a_small = (pair_sm(d, s) || paired_down(d)) ? 0 : 1;
-  set_wide_maps(&dn, 0, h, R, d.F, dn.a_wide, p->wd, nullptr, d.E, d.D, dn.bw_chunks);
+  set_wide_maps(&dn, 0, h, R, d.F, dn.a_wide, p->wd, nullptr, d.el, d.D, dn.bw_chunks);
   set_wide_maps(&dn, 1, hs, d.T, d.S, dn.a_wide, p->sd, nullptr, 1, d.D, dn.bw_chunks);
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
@@ -688,6 +696,8 @@ Dims fp4_dims_of(const moe_nvfp4_params* p) {
   d.E = p->num_experts ? p->num_experts : MOE_NUM_EXPERTS;
   d.F = p->expert_dim ? p->expert_dim : MOE_EXPERT_DIM;
   d.S = p->hidden_dim ? p->hidden_dim : MOE_HIDDEN_DIM;
+  d.e0 = 0;
+  d.el = d.E;
   return d;
 }
 
@@ -734,7 +744,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 0, 0);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 0, 0, 0, d.E);
     MOE_TRY(ls_.done(le_));
   }
   {
@@ -820,7 +830,11 @@ namespace {
 // Scratch of moe_route_noalloc: one fixed array per device that loads this
 // library, held until the process exits. It carries the router's split-K
 // partial logits and the 32-token expert bitmasks of a single call.
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+// Sized for moe_route's own split of the reduction at every T <= 4096: the
+// router runs at most kSmCountHint (token tile, split) CTAs, so splits x T <=
+// 148 x 128 and the partials take <= 148 * 128 * 128 * 4 B = 9.25 MiB, plus
+// <= 64 KiB of bitmasks.
+constexpr size_t kNoAllocScratchBytes = size_t(10) << 20;  // 10 MiB
 constexpr int kNoAllocMaxTokens = 4096;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 uint8_t* g_noalloc_base[kMaxDevices] = {};
@@ -1065,13 +1079,16 @@ moe_status moe_route(const moe_params* p, int32_t* idx, float* w, void* stream) 
   if (d.T == 0) return MOE_OK;
   if (!p->x || !p->w_router || !idx || !w) return MOE_ERR_INVALID_ARG;
   if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned4(idx) || !aligned4(w)) return MOE_ERR_ALIGNMENT;
-  if (p->router_bias && !aligned4(p->router_bias)) return MOE_ERR_ALIGNMENT;
+  if ((p->router_bias && !aligned4(p->router_bias)) || (p->logits_out && !aligned4(p->logits_out)))
+    return MOE_ERR_ALIGNMENT;
   DeviceState* s = nullptr;
   MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
   const Layout L = make_layout(d);
   uint8_t* ws = nullptr;
   MOE_TRY(resolve_workspace(p, s, L, &ws));
-  return enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream));
+  return enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream),
+                       p->logits_out);
 }
 
 moe_status moe_permute(const moe_params* p, const int32_t* idx, int32_t* cnt, int32_t* off, int32_t* row_of,
@@ -1144,12 +1161,28 @@ const char* moe_status_string(moe_status st) {
 
 int moe_last_launch_count(void) { return t_launches; }
 
+moe_status moe_round_bf16(const float* in, void* out, size_t n, void* stream) {
+  t_launches = 0;
+  if (n == 0) return MOE_OK;
+  if (!in || !out || n % 8) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(out)) return MOE_ERR_ALIGNMENT;
+  const uintptr_t ib = reinterpret_cast<uintptr_t>(in), ob = reinterpret_cast<uintptr_t>(out);
+  if (ib < ob + n * 2 && ob < ib + n * 4) return MOE_ERR_INVALID_ARG;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n8 = n / 8;
+  const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, static_cast<size_t>(s->sm_count) * 8));
+  LaunchScope ls_(kKCombine, st);
+  return ls_.done(launch_k(round_bf16_kernel, blocks, 256, 0, st, in, n8, static_cast<__nv_bfloat16*>(out)));
+}
+
 moe_status moe_block_forward_hostio(const moe_params* p, const void* x_host, void* out_host, void* stream) {
   t_launches = 0;
   Dims d;
   MOE_TRY(check_block_args(p, &d));
   if (d.T == 0) return MOE_OK;
-  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (!x_host || !out_host || !p->out) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = static_cast<size_t>(d.T) * d.D * 2;
   if (cudaMemcpyAsync(const_cast<void*>(p->x), x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
@@ -1208,22 +1241,24 @@ moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* 
   if (d.T > kNoAllocMaxTokens) return MOE_ERR_WORKSPACE;
   if (!p->x || !p->w_router || !idx || !w) return MOE_ERR_INVALID_ARG;
   if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned4(idx) || !aligned4(w)) return MOE_ERR_ALIGNMENT;
-  if (p->router_bias && !aligned4(p->router_bias)) return MOE_ERR_ALIGNMENT;
+  if ((p->router_bias && !aligned4(p->router_bias)) || (p->logits_out && !aligned4(p->logits_out)))
+    return MOE_ERR_ALIGNMENT;
   DeviceState* s = nullptr;
   MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
   uint8_t* scratch = nullptr;
   MOE_TRY(noalloc_base(&scratch));
-  // Same kernels and split of the reduction as moe_route, with the partial
-  // logits and bitmasks placed in the fixed array; the split shrinks only if
-  // the partials would not fit (the bitmasks are cleared by the router kernel).
+  // Same kernels and the same split of the reduction as moe_route (so the same
+  // summation order and results), with the partial logits and bitmasks placed
+  // in the fixed array (the bitmasks are cleared by the router kernel).
   Layout L = make_layout(d);
   const size_t mask_bytes = align_up(static_cast<size_t>(L.nchunks) * d.E * 4, kAlign);
-  auto partial_bytes = [&](int ns) { return align_up(static_cast<size_t>(ns) * d.T * d.E * 4, kAlign); };
-  while (L.nsplit > 1 && partial_bytes(L.nsplit) + mask_bytes > kNoAllocScratchBytes) --L.nsplit;
-  if (partial_bytes(L.nsplit) + mask_bytes > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+  const size_t partial_bytes = align_up(static_cast<size_t>(L.nsplit) * d.T * d.E * 4, kAlign);
+  if (partial_bytes + mask_bytes > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
   L.partial = 0;
-  L.masks = partial_bytes(L.nsplit);
-  return enqueue_route(d, L, scratch, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream));
+  L.masks = partial_bytes;
+  return enqueue_route(d, L, scratch, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream),
+                       p->logits_out);
 }
 
 moe_status moe_nvfp4_weight_bytes(int groups, int K, int N, size_t* q_bytes, size_t* sf_bytes) {
@@ -1289,6 +1324,32 @@ size_t moe_nvfp4_workspace_bytes(const moe_nvfp4_params* p) {
   return make_fp4_layout(d).total;
 }
 
+moe_status moe_nvfp4_workspace_layout(const moe_nvfp4_params* p, moe_nvfp4_ws_layout* out) {
+  if (!p || !out) return MOE_ERR_INVALID_ARG;
+  const Dims d = fp4_dims_of(p);
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  const Fp4Layout F = make_fp4_layout(d);
+  out->total_bytes = F.total;
+  out->xq_perm = F.xq_perm;
+  out->xsf_perm = F.xsf_perm;
+  out->xq_tok = F.xq_tok;
+  out->xsf_tok = F.xsf_tok;
+  out->hq = F.hq;
+  out->hsf = F.hsf;
+  out->hsq = F.hsq;
+  out->hssf = F.hssf;
+  out->y = F.y;
+  out->s = F.s;
+  out->idx = F.r.idx;
+  out->w = F.r.w;
+  out->cnt = F.r.cnt;
+  out->off = F.r.off;
+  out->row_of = F.r.row_of;
+  out->routed_rows = F.r_pad;
+  out->token_rows = F.t_pad;
+  return MOE_OK;
+}
+
 moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream) {
   t_launches = 0;
   Dims d;
@@ -1311,17 +1372,21 @@ moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream) {
   return enqueue_block_fp4(p, d, F, ws, s, static_cast<cudaStream_t>(stream));
 }
 
-moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream) {
+moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, float* scales, void* stream) {
   t_launches = 0;
   Dims d;
   MOE_TRY(check_block_args(p, &d));
-  if (!amax || !p->workspace) return MOE_ERR_INVALID_ARG;
-  if (!aligned4(amax)) return MOE_ERR_ALIGNMENT;
+  if (!amax || !scales || !p->workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned4(amax) || !aligned4(scales)) return MOE_ERR_ALIGNMENT;
+  if (amax < scales + 3 && scales < amax + 3) return MOE_ERR_INVALID_ARG;
   DeviceState* s = nullptr;
   MOE_TRY(device_state(&s));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(amax, 0, 3 * sizeof(float), st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (d.T == 0) return MOE_OK;
+  if (d.T == 0) {
+    LaunchScope ls_(kKTensorScale, st);
+    return ls_.done(launch_k(tensor_scale_kernel, 1, 32, 0, st, reinterpret_cast<const uint32_t*>(amax), scales, 3));
+  }
   if (!encode_fn()) return MOE_ERR_CUDA;
   const Layout L = make_layout(d);
   uint8_t* ws = nullptr;
@@ -1337,7 +1402,9 @@ moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, void* stream) {
                                      ns[i], reinterpret_cast<uint32_t*>(amax) + i);
     MOE_TRY(ls_.done(le_));
   }
-  return MOE_OK;
+  // the three tensor scales G = 448 * 6 / amax (1 for an all-zero tensor)
+  LaunchScope ls_(kKTensorScale, st);
+  return ls_.done(launch_k(tensor_scale_kernel, 1, 32, 0, st, reinterpret_cast<const uint32_t*>(amax), scales, 3));
 }
 
 size_t moe_dense_workspace_bytes(const moe_dense_params* p) {

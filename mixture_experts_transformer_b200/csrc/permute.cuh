@@ -20,6 +20,8 @@
 namespace moe {
 
 constexpr int kScanThreads = 1024;
+// row_of of a (token, slot) whose expert belongs to another expert shard
+constexpr int32_t kRowNotLocal = -1;
 constexpr int kScanSegs = kScanThreads / 128;
 
 struct TileCounts {
@@ -52,6 +54,11 @@ __global__ void build_masks_kernel(const int32_t* __restrict__ idx, int T, int k
 // shared-MLP tiles first (problem 1), then expert tiles (problem 0) expert by
 // expert, column tile, then row tile, so CTAs that run at the same time read
 // the same weight columns and share them through L2.
+//
+// An expert shard (expert parallelism) owns experts [e_begin, e_begin +
+// e_count): only they get routed rows and tiles (their cnt is the real count,
+// every other expert's is 0), and a tile's weight group is the expert's index
+// within the shard. The whole block is e_begin = 0, e_count = E.
 __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t* __restrict__ masks, int nchunks,
                                                                   int T, int E, int F, int S, int D,
                                                                   int32_t* __restrict__ base,
@@ -60,7 +67,8 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
                                                                   Tile* __restrict__ tiles_gu,
                                                                   Tile* __restrict__ tiles_dn,
                                                                   TileCounts* __restrict__ counts, int padded,
-                                                                  int dn_cols, int pair_gu, int pair_dn) {
+                                                                  int dn_cols, int pair_gu, int pair_dn,
+                                                                  int e_begin, int e_count) {
   __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
   __shared__ int s_mtoff[129];
@@ -71,8 +79,9 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   const int seg = threadIdx.x >> 7;
   const int c0 = static_cast<int>((static_cast<long long>(seg) * nchunks) / kScanSegs);
   const int c1 = static_cast<int>((static_cast<long long>(seg + 1) * nchunks) / kScanSegs);
+  const bool local = e >= e_begin && e < e_begin + e_count && e < E;
   int part = 0;
-  if (e < E) {
+  if (local) {
 #pragma unroll 8
     for (int c = c0; c < c1; ++c) part += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
   }
@@ -125,17 +134,17 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   // first routed row of expert e: packed (bf16 path) or padded to whole
   // 128-row tiles (NVFP4 path: every tile starts on a scale-atom boundary)
   const int row_base = padded ? s_mtoff[e] * kBM : s_off[e];
-  if (e < E) {
+  if (local) {
     int run = row_base + s_seg[seg][e];
 #pragma unroll 8
     for (int c = c0; c < c1; ++c) {
       base[static_cast<size_t>(c) * E + e] = run;
       run += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
     }
-    if (seg == 0) {
-      cnt_out[e] = c_e;
-      off_out[e] = s_off[e];
-    }
+  }
+  if (e < E && seg == 0) {
+    cnt_out[e] = c_e;
+    off_out[e] = s_off[e];
   }
   if (threadIdx.x == 0) off_out[E] = s_off[E];
 
@@ -171,7 +180,8 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
       const int nt = i / pt, m = (i % pt) * mstep;
       const int rb = padded ? s_mtoff[ex] * kBM : s_off[ex];
       const int r1 = pair ? max(0, min(kBM, ce - (m + 1) * kBM)) : 0;
-      tiles[n_sh + f] = Tile{ex, rb + m * kBM, min(kBM, ce - m * kBM), nt * cw, rb + (m + 1) * kBM, r1, 0, 0};
+      tiles[n_sh + f] =
+          Tile{ex - e_begin, rb + m * kBM, min(kBM, ce - m * kBM), nt * cw, rb + (m + 1) * kBM, r1, 0, 0};
     }
     return n_sh + n_e;
   };
@@ -270,6 +280,8 @@ __global__ void __launch_bounds__(256) round_bf16_kernel(const float* __restrict
 // One warp per (token, slot): its routed row from the bitmasks; lane 0 writes
 // row_of / token_of, and (when x is given) the warp copies x[t] into
 // x_perm[row] with 16-byte vectors, so the GEMM's A tiles are plain boxes.
+// Slots whose expert lies outside the shard [e_begin, e_begin + e_count) get
+// row_of = kRowNotLocal and no row.
 __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __restrict__ idx,
                                                             const uint32_t* __restrict__ masks,
                                                             const int32_t* __restrict__ base, int T, int k, int E,
@@ -277,7 +289,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
                                                             int32_t* __restrict__ row_of,
                                                             int32_t* __restrict__ token_of,
                                                             __nv_bfloat16* __restrict__ x_perm, long long rows,
-                                                            uint32_t* __restrict__ err) {
+                                                            uint32_t* __restrict__ err, int e_begin, int e_count) {
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const long long R = static_cast<long long>(T) * k;
@@ -286,6 +298,10 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
     const int t = static_cast<int>(a / k);
     const int e = __ldg(idx + a);
     if (e < 0 || e >= E) continue;  // reported by build_masks_kernel
+    if (e < e_begin || e >= e_begin + e_count) {
+      if (lane == 0) row_of[a] = kRowNotLocal;
+      continue;
+    }
     const size_t cw = static_cast<size_t>(t / kMaskTokens) * E + e;
     const uint32_t below = __ldg(masks + cw) & ((1u << (t & (kMaskTokens - 1))) - 1u);
     const int row = __ldg(base + cw) + __popc(below);
@@ -308,6 +324,8 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int32_t* __res
 // out[t] = RNE_bf16(s[t] + w[t,0] y[row_of[t,0]] + ... + w[t,k-1] y[row_of[t,k-1]]),
 // accumulated in fp32 in slot order (deterministic, no atomics). Grid (T,
 // dsplit): CTA (t, q) handles the q-th slice of the row's 8-column vectors.
+// Slots marked kRowNotLocal (an expert shard's foreign experts) are left out;
+// out (bf16) may be null when only out_f32 is wanted.
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ s, const __nv_bfloat16* __restrict__ y,
                                                      const int32_t* __restrict__ row_of,
                                                      const float* __restrict__ w, int T, int k, int D, int rows,
@@ -315,20 +333,31 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
                                                      uint32_t* __restrict__ err) {
   __shared__ int s_row[128];
   __shared__ float s_w[128];
+  __shared__ int s_k;
   pdl_wait_then_release();
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < k; j += blockDim.x) {
-    int r = row_of[static_cast<size_t>(t) * k + j];
-    float wj = w[static_cast<size_t>(t) * k + j];
-    if (r < 0 || r >= rows) {  // a routed row outside y: report, never address it
-      atomicOr(err, kErrBadIndex);
-      r = 0;
-      wj = 0.f;
-    }
-    s_row[j] = r;
-    s_w[j] = wj;
+    s_row[j] = row_of[static_cast<size_t>(t) * k + j];
+    s_w[j] = w[static_cast<size_t>(t) * k + j];
   }
   __syncthreads();
+  if (threadIdx.x == 0) {  // keep the token's slots with a routed row here, in slot order
+    int kk = 0;
+    for (int j = 0; j < k; ++j) {
+      const int r = s_row[j];
+      if (r == kRowNotLocal) continue;
+      if (r < 0 || r >= rows) {  // a routed row outside y: report, never address it
+        atomicOr(err, kErrBadIndex);
+        continue;
+      }
+      s_row[kk] = r;
+      s_w[kk] = s_w[j];
+      ++kk;
+    }
+    s_k = kk;
+  }
+  __syncthreads();
+  k = s_k;
   const int nvec = D >> 3;
   const int per = (nvec + gridDim.y - 1) / gridDim.y;
   const int v0 = blockIdx.y * per, v1 = min(nvec, v0 + per);
@@ -357,12 +386,14 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, __bfloat162float(yb[i]), acc[i]);
     }
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * D)[v] = o;
+    if (out) {
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * D)[v] = o;
+    }
     if (out_f32) {
       float4* op = reinterpret_cast<float4*>(out_f32 + static_cast<size_t>(t) * D) + 2 * v;
       op[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);

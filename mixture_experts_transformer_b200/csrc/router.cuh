@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_kernel(const __g
 
 // One warp per token: sum the split partials in split order, add the bias,
 // pick the k largest (ties: lower index), softmax over them, set the token's
-// bits in the expert bitmasks. Lane l holds experts l, l+32, l+64, l+96.
+// bits in the expert bitmasks; with logits_out, also write the summed logits
+// (bias included) as a debug output. Lane l holds experts l, l+32, l+64, l+96.
 // ALL_SPLITS (small batches, many splits of the router's reduction): every
 // split's loads are in flight at once, one memory round trip instead of one
 // per four splits; large batches keep the leaner loop, whose lower register
@@ -214,7 +215,8 @@ __global__ void __launch_bounds__(kTopkWarps * 32) router_topk_kernel(const floa
                                                                      const float* __restrict__ bias, int T, int E,
                                                                      int nsplit, int k, int32_t* __restrict__ idx,
                                                                      float* __restrict__ wts,
-                                                                     uint32_t* __restrict__ masks) {
+                                                                     uint32_t* __restrict__ masks,
+                                                                     float* __restrict__ logits_out) {
   pdl_wait_then_release();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kTopkWarps + (threadIdx.x >> 5);
@@ -267,6 +269,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) router_topk_kernel(const floa
     float v = -INFINITY;
     if (e < E) {
       v = l[q] + (bias ? bias[e] : 0.f);
+      if (logits_out) logits_out[static_cast<size_t>(t) * E + e] = v;
       if (isnan(v)) v = -INFINITY;  // a NaN never wins, so the k winners stay valid experts
     }
     l[q] = v;

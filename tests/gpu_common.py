@@ -29,13 +29,14 @@ OUT_TOL = 1e-2
 BF16_SLACK = 1.25
 ACC_SLACK = 2e-3
 GAP = 1e-4
-# Routing weights. Requiring exact expert sets wherever the oracle's logit gap
-# exceeds GAP presumes the kernel's logits agree with the oracle's to well
-# under GAP; the tensor cores accumulate the router's products in fp32 in their
-# own order, so take LOGIT_TOL = GAP / 4 as that agreement. A logit error of at
-# most d moves the weight softmax(l)_j by at most 2 d w_j (one term from l_j,
-# one from the normaliser), hence the relative bound W_REL.
-LOGIT_TOL = GAP / 4
+# Router logits: measured against the oracle's fp64 logits at the Gemma shapes
+# (test_router_logits_against_oracle, seeded x ~ N(0, 1)): max |err| 9.1e-7 at
+# T = 64 (22 splits of the reduction), 4.0e-6 at T = 4096 and 4.4e-6 at
+# T = 4096 with the Zipf router bias (4 splits: longer sums inside the tensor
+# cores' fp32 accumulators). LOGIT_TOL keeps a margin of ~2.3x over the largest.
+# A logit error of at most d moves the weight softmax(l)_j by at most 2 d w_j
+# (one term from l_j, one from the normaliser), hence the relative bound W_REL.
+LOGIT_TOL = 1e-5
 W_REL = 2 * LOGIT_TOL
 
 SMALL = inputs.Dims(embed_dim=256, num_experts=16, expert_dim=192, hidden_dim=320)
@@ -104,14 +105,19 @@ def _rne_bf16_f64(a):
     return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).double().numpy()
 
 
-def bf16_storage_cost(xs, w_host, idx, wts):
-    """max |out(h, y, hs rounded to bf16) - out(exact)| for the given routing (CPU, float64)."""
+def bf16_storage_cost(xs, w_host, idx, wts, hidden=None, experts=None):
+    """max |out(h, y, hs rounded to bf16) - out(exact)| for the given routing (CPU,
+    float64). hidden = (h0, h1) and experts = (e0, e1) restrict it to an expert
+    shard's part: its slice of the shared MLP's hidden units and its experts."""
     x = mo.f64(xs)
-    hs = mo.geglu_hidden(x, w_host.sg, w_host.su)
-    sd = mo.f64(w_host.sd)
+    h0, h1 = hidden if hidden is not None else (0, w_host.sg.shape[1])
+    hs = mo.geglu_hidden(x, w_host.sg[:, h0:h1], w_host.su[:, h0:h1])
+    sd = mo.f64(w_host.sd[h0:h1])
     exact = hs @ sd
     rounded = _rne_bf16_f64(hs) @ sd  # the shared hidden rows are stored in bf16 too
     for e in np.unique(idx):
+        if experts is not None and not experts[0] <= e < experts[1]:
+            continue
         tok, slot = np.nonzero(idx == e)
         h = mo.geglu_hidden(x[tok], w_host.wg[e], w_host.wu[e])
         wd = mo.f64(w_host.wd[e])
@@ -124,14 +130,18 @@ def bf16_storage_cost(xs, w_host, idx, wts):
 def check_block_output(w_host, x_bits, res, k, bias=None, tokens=None, derived_tol=False):
     """Oracle on (a subset of) tokens: routing per check_routing, output within
     tolerance given the GPU's own routing, and out == RNE(out_f32) exactly.
-    derived_tol=False: the 1e-2 * RMS bound (Gemma shapes); True: the bound
-    derived from the bf16 storage of h and y (reduced shapes)."""
+    derived_tol=False: the 1e-2 * RMS bound; True: the larger of that and the
+    bound derived from the bf16 storage of h, hs and y - at reduced shapes,
+    where the routed branch weighs more, and for samples of hundreds to
+    thousands of Gemma-shape tokens, whose largest elements' rounding alone
+    passes 1e-2 * RMS (measured at T = 16384 with the Zipf bias, 1971 tokens:
+    GPU error 1.073% of RMS, the emulated roundings 1.076%)."""
     tok = np.arange(x_bits.shape[0]) if tokens is None else np.asarray(tokens)
     xs = x_bits[tok]
     idx = to_np(res.idx)[tok]
     wts = to_np(res.w)[tok]
-    ref = mo.moe_block(xs, *w_args(w_host), top_k=k, bias=bias)
-    check_routing(ref["logits"], ref["idx"], ref["w"], idx, wts, k)
+    ref_idx, ref_w, ref_logits = mo.route(xs, w_host.w_router, k, bias)
+    check_routing(ref_logits, ref_idx, ref_w, idx, wts, k)
     ref_g = mo.moe_block(xs, *w_args(w_host), routing=(idx, wts))
     out32 = to_np(res.out_f32)[tok].astype(np.float64)
     rms = np.sqrt(np.mean(ref_g["out"] ** 2))
@@ -142,6 +152,27 @@ def check_block_output(w_host, x_bits, res, k, bias=None, tokens=None, derived_t
     assert err <= bound, (err, rms, err / rms, bound / rms)
     np.testing.assert_array_equal(bf16_to_f32(res.out)[tok], rne_bf16(to_np(res.out_f32)[tok]))
     return err / rms
+
+
+def ws_view(ws: torch.Tensor, offset: int, count: int, dtype) -> torch.Tensor:
+    """count elements of dtype at a byte offset of a uint8 workspace."""
+    size = torch.tensor([], dtype=dtype).element_size()
+    return ws[offset : offset + count * size].view(dtype)
+
+
+def tile_covering_tokens(ws: torch.Tensor, lay, T: int, k: int, num_experts: int, block_rows: int = 128):
+    """Tokens of the first and last routed row of every 128-row block of every
+    expert (rows of expert e start at off[e]), read from the GPU's own
+    permutation: comparing them with the oracle touches every GEMM row tile."""
+    token_of = to_np(ws_view(ws, lay.token_of, T * k, torch.int32))
+    off = to_np(ws_view(ws, lay.off, num_experts + 1, torch.int32))
+    toks = set()
+    for e in range(num_experts):
+        for r0 in range(int(off[e]), int(off[e + 1]), block_rows):
+            r1 = min(r0 + block_rows, int(off[e + 1])) - 1
+            toks.add(int(token_of[r0]))
+            toks.add(int(token_of[r1]))
+    return np.array(sorted(toks), dtype=np.int64)
 
 
 def skip_unless(cond, why):

@@ -96,3 +96,33 @@ def test_host_validation(lib):
     assert f(p) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_block_forward_ex(None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_timeout_probe(0, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_expert_shard_validation(lib):
+    """Expert-shard fields and the optional bf16 output, checked on the host."""
+    f = lambda p: lib.moe_block_forward_ex(ctypes.byref(p), None)  # noqa: E731
+    p = _params(expert_begin=120, expert_count=16)  # past the 128 experts
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params(expert_begin=-1, expert_count=4)
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params(out=None)  # no output at all
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params(out=1 << 40 | 8)  # misaligned bf16 output
+    assert f(p) == B.MOE_ERR_ALIGNMENT
+    # a shard's output is a partial sum: no post-norm, no residual
+    p = _params(expert_begin=64, expert_count=64, out=None, out_f32=1 << 41, norm_post=16)
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    p = _params(expert_begin=0, expert_count=64, residual=True)
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+    # fp32 output alone, without the bf16 one, but with the post-norm: refused too
+    p = _params(out=None, out_f32=1 << 41, norm_post=16)
+    assert f(p) == B.MOE_ERR_INVALID_ARG
+
+
+def test_round_bf16_validation(lib):
+    f = lib.moe_round_bf16
+    assert f(None, None, 0, None) == B.MOE_OK  # nothing to do
+    assert f(None, 16, 8, None) == B.MOE_ERR_INVALID_ARG
+    assert f(16, 1 << 20, 12, None) == B.MOE_ERR_INVALID_ARG  # n not a multiple of 8
+    assert f(20, 1 << 20, 8, None) == B.MOE_ERR_ALIGNMENT
+    assert f(1 << 20, (1 << 20) + 16, 8, None) == B.MOE_ERR_INVALID_ARG  # overlap

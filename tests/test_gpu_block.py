@@ -11,7 +11,9 @@ from gpu_common import (
     check_routing,
     device_weights,
     require_gpu,
+    LOGIT_TOL,
     run_block,
+    tile_covering_tokens,
     to_np,
     w_args,
     weights,
@@ -29,6 +31,25 @@ def _gpu():
 
 
 # ------------------------------------------------------------------ router
+
+
+@pytest.mark.parametrize("T,skew", [(64, False), (4096, False), (4096, True)])
+def test_router_logits_against_oracle(T, skew):
+    """The router's fp32 logits (tensor-core products of bf16 values, exact in
+    fp32, accumulated in the hardware's order, split partials summed in split
+    order) against the oracle's fp64 logits, element by element. The measured
+    error sets the routing tolerance LOGIT_TOL of the other tests."""
+    w = weights()
+    dw = device_weights()
+    bias = inputs.zipf_router_bias() if skew else None
+    x_bits = inputs.make_x(T, seed=90 + T)
+    res = run_block(dw, x_bits, bias=bias)
+    ref = mo.router_logits(x_bits, w.w_router, bias)
+    got = to_np(res.logits).astype(np.float64)
+    err = np.abs(got - ref)
+    print(f"router logits T={T} skew={skew}: max |err| {err.max():.3e}, "
+          f"99.9th pct {np.quantile(err, 0.999):.3e}, |logit| max {np.abs(ref).max():.2f}")
+    assert err.max() <= LOGIT_TOL, err.max()
 
 
 @pytest.mark.parametrize("T", [1, 7, 64, 257])
@@ -187,29 +208,42 @@ def test_block_gemma(T):
 
 
 def test_block_gemma_prefill_sampled():
-    """T = 4096 in the benchmark's launch configuration; 48 sampled tokens
-    against the oracle (tokens are independent in the block)."""
+    """T = 4096 in the benchmark's launch configuration (paired gate|up, down
+    on SM pairs): 512 seeded random tokens plus the first and last token of
+    every 128-row block of every expert against the oracle (tokens are
+    independent in the block), so every row tile of both GEMMs is compared."""
     T = 4096
     w = weights()
     dw = device_weights()
     x_bits = inputs.make_x(T)
-    res = run_block(dw, x_bits)
-    check_block_output(w, x_bits, res, 8, tokens=inputs.sample_tokens(T, 48))
+    ws, lay = block.workspace_for(inputs.GEMMA4_26B_A4B, T)
+    res = run_block(dw, x_bits, workspace=ws)
     cnt = to_np(res.cnt)
     assert cnt.sum() == 8 * T and cnt.min() > 0
+    tiles = tile_covering_tokens(ws, lay, T, 8, inputs.NUM_EXPERTS)
+    tokens = np.union1d(inputs.sample_tokens(T, 512), tiles)
+    assert len(tokens) >= 512
+    check_block_output(w, x_bits, res, 8, tokens=tokens, derived_tol=True)
 
 
-def test_block_gemma_skewed_sampled():
-    """T = 16384 with the Zipf(1.1) router bias: a few experts take most rows."""
+def test_block_gemma_skewed_every_tile():
+    """T = 16384 with the Zipf(1.1) router bias: a few experts take most rows
+    (the hottest holds almost every token, ~128 row blocks). The sample is the
+    first and last token of every 128-row block of every expert, read from the
+    GPU's own permutation, so every tile of the long tail and of the hot
+    expert is compared with the oracle."""
     T = 16384
     w = weights()
     dw = device_weights()
     bias = inputs.zipf_router_bias()
     x_bits = inputs.make_x(T)
-    res = run_block(dw, x_bits, bias=bias)
+    ws, lay = block.workspace_for(inputs.GEMMA4_26B_A4B, T)
+    res = run_block(dw, x_bits, bias=bias, workspace=ws)
     cnt = np.sort(to_np(res.cnt))[::-1]
     assert cnt[:13].sum() > 0.5 * 8 * T
-    check_block_output(w, x_bits, res, 8, bias=bias, tokens=inputs.sample_tokens(T, 32))
+    tokens = tile_covering_tokens(ws, lay, T, 8, inputs.NUM_EXPERTS)
+    assert len(tokens) >= 512
+    check_block_output(w, x_bits, res, 8, bias=bias, tokens=tokens, derived_tol=True)
 
 
 def test_deterministic():
