@@ -54,6 +54,14 @@ WORKLOADS = {
         layers=30,
         desc="30 Gemma-4-26B-A4B MoE blocks in NVFP4 (group 16, e4m3 scales), RMSNorm between blocks, T=2048",
     ),
+    "decode_sfp8": dict(
+        T=64, bias=False, bound="hbm", wq="sfp8",
+        desc="Gemma-4-26B-A4B MoE block, T=64 tokens, SFP8 weight-only expert and shared Linears, bf16 activations",
+    ),
+    "decode_q4_0": dict(
+        T=64, bias=False, bound="hbm", wq="q4_0",
+        desc="Gemma-4-26B-A4B MoE block, T=64 tokens, Q4_0 weight-only expert and shared Linears, bf16 activations",
+    ),
     "e4b_dense_decode": dict(
         T=64, bias=False, bound="hbm", dense=True,
         desc="Gemma-4-E4B dense GeGLU FFN (embed 2560, hidden 10240), T=64 tokens, bf16",
@@ -791,6 +799,9 @@ def run_reference(args, world, rank):
 
     wl = WORKLOADS[args.workload]
     T = wl["T"]
+    if wl.get("wq"):
+        return {"impl": "reference", "unavailable": "the oracle's weight-only block quantises every touched expert's "
+                "weights per call (minutes of host time per step), beyond a bounded step"}
     if args.workload == "nvfp4_stack":
         # one oracle step re-quantises the weights of every touched expert
         # (~126 x 3 matrices per layer, minutes per layer on the host)
@@ -1022,6 +1033,158 @@ def run_dense(args, world, rank, local):
     return res
 
 
+def wq_weight_bytes(fmt: str, K: int, N: int) -> int:
+    """Bytes of one [K, N] Linear in the library's weight-only layout (rows padded to 128)."""
+    blk = 8192 if fmt == "sfp8" else 4608
+    return ((N + 127) // 128) * (K // 64) * blk
+
+
+def run_wq(args, world, rank, local):
+    """One step = the block with weight-only SFP8 / Q4_0 weights over T tokens."""
+    import torch
+
+    from mixture_experts_transformer_b200 import binding as B
+    from mixture_experts_transformer_b200 import block, build, inputs
+
+    if rank == 0:
+        build.build()
+    barrier(world)
+    B.lib()
+    torch.cuda.set_device(local)
+    wl = WORKLOADS[args.workload]
+    T, fmt = wl["T"], wl["wq"]
+    ww = block.quantize_wq(gen_weights_gpu(seed=0), fmt)
+    torch.cuda.synchronize()
+    gx = torch.Generator(device="cuda").manual_seed(1 + rank)
+    x = torch.empty((T, D), dtype=torch.float32, device="cuda").normal_(0.0, 1.0, generator=gx).to(torch.bfloat16)
+    out = torch.empty((T, D), dtype=torch.bfloat16, device="cuda")
+    p0 = block.wq_params(ww, T, None, None)
+    ws = torch.empty(B.moe_wq_workspace_bytes(p0), dtype=torch.uint8, device="cuda")
+    p = block.wq_params(ww, T, x, out, workspace=ws)
+    stream = torch.cuda.current_stream()
+    dbg = block.forward_wq(ww, x, debug=True, workspace=ws)
+    torch.cuda.synchronize()
+    cnt = dbg.cnt.cpu().numpy()
+    touched = int((cnt > 0).sum())
+    if B.moe_get_device_status() != B.MOE_OK:
+        raise RuntimeError("device status after the debug pass")
+    for _ in range(max(args.warmup, 3)):
+        B.check(B.moe_block_forward_wq(p, stream), "wq")
+    torch.cuda.synchronize()
+    launches = B.moe_last_launch_count()
+    B.moe_profile_begin()
+    for _ in range(min(args.steps, 50)):
+        B.check(B.moe_block_forward_wq(p, stream), "wq")
+    torch.cuda.synchronize()
+    breakdown = B.moe_profile_end()
+    dominant = max(breakdown, key=lambda k: breakdown[k][0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            B.check(B.moe_block_forward_wq(p, stream), "wq")
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = reduce_max(e0.elapsed_time(e1), world)
+    agg = aggregate(T, args.steps, ms, world)
+    B.moe_profile_begin([dominant])
+    for _ in range(args.steps):
+        B.check(B.moe_block_forward_wq(p, stream), "wq")
+    torch.cuda.synchronize()
+    per_kernel = B.moe_profile_end()
+    if B.moe_get_device_status() != B.MOE_OK:
+        raise RuntimeError("device status after the timed region")
+    # end to end: pinned host x in, host out back, through the public call
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    pe = block.wq_params(ww, T, x_dev, out, workspace=ws)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        B.check(B.moe_block_forward_wq(pe, stream), "wq")
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(t0.elapsed_time(t1), world)
+    barrier(world)
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    step_ms = agg["ms_per_step"]
+    R = T * K_TOP
+    e_gu = 2 * wq_weight_bytes(fmt, D, F)
+    e_dn = wq_weight_bytes(fmt, F, D)
+    sh_gu, sh_dn = 2 * wq_weight_bytes(fmt, D, S), wq_weight_bytes(fmt, S, D)
+    if dominant == "grouped_gemm_gateup":
+        byts = touched * e_gu + sh_gu + (R + T) * D * 2 + (R * F + T * S) * 2
+    elif dominant == "grouped_gemm_down":
+        byts = touched * e_dn + sh_dn + (R * F + T * S) * 2 + R * D * 2 + T * D * 4
+    else:
+        byts, _ = algorithmic(dominant, T, touched, cnt)
+    dom_ms = per_kernel[dominant][0] / per_kernel[dominant][1]
+    weight_bytes = touched * (e_gu + e_dn) + sh_gu + sh_dn + ROUTER_BYTES
+    return {
+        "metric": METRIC,
+        "value": agg["value"],
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": f"{fmt} weights (weight-only), bf16 activations, fp32 accumulate",
+        "data": "synthetic: seeded N(0,0.02) random-init weights of the published shapes, quantised by the library",
+        "config": {
+            "workload": wl["desc"],
+            "tokens_per_gpu": T,
+            "global_batch": T * world,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": dominant,
+            "achieved": byts / (dom_ms / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"],
+            "peak_source": f"{peaks['source']} hbm_gbs",
+            "unit": "GB/s",
+            "frac": byts / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "traffic": None,
+            "algorithmic_bytes": byts,
+            "kernel_ms": dom_ms,
+        },
+        "block_roofline": {
+            "hbm_touched_weights_gbs": weight_bytes / (step_ms / 1e3) / 1e9,
+            "hbm_frac": weight_bytes / (step_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "touched_experts": touched,
+            "weight_bytes": weight_bytes,
+        },
+        "kernels_ms_per_launch": {k: v[0] / v[1] for k, v in breakdown.items()},
+        "gpu_launches": launches * args.steps,
+        "e2e": {
+            "value": T * args.steps * world / (e2e_ms / 1e3),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": T * D * 2,
+            "d2h_bytes_per_step": T * D * 2,
+        },
+        "clocks": clocks.report(),
+    }
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args.gpus)
@@ -1032,6 +1195,8 @@ def main():
             res = run_stack(args, world, rank, local)
         elif WORKLOADS[args.workload].get("dense"):
             res = run_dense(args, world, rank, local)
+        elif WORKLOADS[args.workload].get("wq"):
+            res = run_wq(args, world, rank, local)
         else:
             res = run_ours(args, world, rank, local)
         if rank == 0 and res is not None:

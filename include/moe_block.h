@@ -399,6 +399,85 @@ moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream);
  */
 moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, float* scales, void* stream);
 
+/* --------------------------------------------- weight-only SFP8 / Q4_0
+ *
+ * The pages give a whole-model footprint for two more weight formats, SFP8
+ * and Q4_0 (Gemma-4-26B-A4B record, "MEMORY IS SET BY TOTAL, NOT ACTIVE":
+ * 57.7 GB bf16, 28.8 GB at SFP8, 14.4 GB at Q4_0), and print neither format.
+ * Readings (weight-only: every expert and shared Linear weight quantised
+ * along its input dimension K, each matrix on its own; router and
+ * activations stay bf16):
+ *   SFP8: sign bit and a 7-bit magnitude code m - 0 is zero, m in [1, 63] is
+ *         (1 + (m & 3)/4) 2^((m >> 2) - 23), m in [64, 127] is
+ *         (1 + (m & 7)/8) 2^(((m >> 3) & 7) - 7) (3 mantissa bits from 2^-7 up,
+ *         2 below, largest 1.875); one fp32 scale S = amax / 1.875 per matrix;
+ *         code = nearest magnitude to |w| / S (ties to the even code,
+ *         saturating) with w's sign; w^ = value * S.
+ *   Q4_0: the ggml block format - blocks of 32 along K, d = (the block's
+ *         first element of largest magnitude, sign kept) / -8 stored as fp16,
+ *         q = min(15, trunc(w / d + 8.5)) in fp32 arithmetic, w^ = (q - 8) d.
+ * The block then computes as the bf16 block on the dequantised weights (h,
+ * y bf16, s fp32, out bf16); SFP8 values are exact in bf16 and the matrix
+ * scale multiplies the fp32 sums, while a Q4_0 weight (q - 8) d is rounded to
+ * bf16 (nearest even) before the tensor cores.
+ *
+ * Storage of G stacked [K, N] Linears (K and N multiples of 64), the
+ * transposed weight in 128-row blocks and 64-deep K blocks:
+ *   SFP8: q [G][ceil(N/128)][K/64][128 rows x 64 code bytes]; scale [G] fp32
+ *   Q4_0: q [G][ceil(N/128)][K/64][128 rows x 32 bytes | 128 rows x 2 fp16 d]
+ *         (element 2j of a row's 64 in the low nibble of byte j; the row's two
+ *         scales cover K 0-31 and 32-63); scale unused (NULL)
+ * Rows past N hold zeros.
+ */
+#define MOE_WFMT_SFP8 1
+#define MOE_WFMT_Q4_0 2
+
+typedef struct moe_wq_linear {
+  const uint8_t* q;
+  const float* scale;
+} moe_wq_linear;
+
+/* Bytes of q for G stacked [K, N] Linears in `format`. */
+moe_status moe_wq_weight_bytes(int format, int groups, int K, int N, size_t* bytes);
+
+/*
+ * Quantise bf16 weights w [groups][K][N] (N contiguous: the bf16 block's
+ * layout) into q (and, SFP8, scale [groups]); caller-owned device buffers of
+ * the sizes above. Deterministic; enqueued on stream.
+ */
+moe_status moe_wq_quantize_weight(int format, const void* w, int groups, int K, int N, uint8_t* q, float* scale,
+                                  void* stream);
+
+/*
+ * One block with weight-only SFP8 or Q4_0 expert and shared Linears. Dims,
+ * x, w_router (bf16), router_bias, out, out_f32, idx_out, w_out, cnt_out and
+ * workspace as in moe_params (workspace: moe_wq_workspace_bytes).
+ */
+typedef struct moe_wq_params {
+  int T;
+  int top_k_experts;
+  int embed_dim;
+  int num_experts;
+  int expert_dim;
+  int hidden_dim;
+  int format;
+  const void* x;
+  const void* w_router;
+  const float* router_bias;
+  moe_wq_linear wg, wu, wd; /* G = num_experts */
+  moe_wq_linear sg, su, sd; /* G = 1 */
+  void* out;
+  float* out_f32;
+  int32_t* idx_out;
+  float* w_out;
+  int32_t* cnt_out;
+  void* workspace;
+  size_t workspace_bytes;
+} moe_wq_params;
+
+size_t moe_wq_workspace_bytes(const moe_wq_params* p);
+moe_status moe_block_forward_wq(const moe_wq_params* p, void* stream);
+
 /* -------------------------------------------------------- dense GeGLU FFN
  *
  * The feed-forward of the dense E4B sibling (gm.nn.Gemma4_E4B

@@ -400,6 +400,79 @@ def moe_nvfp4_calibrate(p: MoeParams, amax, scales, stream=None) -> int:
     return lib().moe_nvfp4_calibrate(ctypes.byref(p), ptr(amax), ptr(scales), stream_handle(stream))
 
 
+# ------------------------------------------------ weight-only SFP8 / Q4_0
+
+WFMT_SFP8 = 1
+WFMT_Q4_0 = 2
+WFORMATS = {"sfp8": WFMT_SFP8, "q4_0": WFMT_Q4_0}
+
+
+class MoeWqLinear(ctypes.Structure):
+    _fields_ = [("q", _vp), ("scale", _vp)]
+
+
+class MoeWqParams(ctypes.Structure):
+    _fields_ = [
+        ("T", ctypes.c_int),
+        ("top_k_experts", ctypes.c_int),
+        ("embed_dim", ctypes.c_int),
+        ("num_experts", ctypes.c_int),
+        ("expert_dim", ctypes.c_int),
+        ("hidden_dim", ctypes.c_int),
+        ("format", ctypes.c_int),
+        ("x", _vp),
+        ("w_router", _vp),
+        ("router_bias", _vp),
+        ("wg", MoeWqLinear),
+        ("wu", MoeWqLinear),
+        ("wd", MoeWqLinear),
+        ("sg", MoeWqLinear),
+        ("su", MoeWqLinear),
+        ("sd", MoeWqLinear),
+        ("out", _vp),
+        ("out_f32", _vp),
+        ("idx_out", _vp),
+        ("w_out", _vp),
+        ("cnt_out", _vp),
+        ("workspace", _vp),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+EXPORTS.update(
+    {
+        "moe_wq_weight_bytes": (
+            ctypes.c_int,
+            [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)],
+        ),
+        "moe_wq_quantize_weight": (
+            ctypes.c_int,
+            [ctypes.c_int, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp],
+        ),
+        "moe_wq_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(MoeWqParams)]),
+        "moe_block_forward_wq": (ctypes.c_int, [ctypes.POINTER(MoeWqParams), _vp]),
+    }
+)
+
+
+def moe_wq_weight_bytes(fmt: int, groups: int, K: int, N: int) -> int:
+    n = ctypes.c_size_t()
+    check(lib().moe_wq_weight_bytes(fmt, groups, K, N, ctypes.byref(n)), "moe_wq_weight_bytes")
+    return n.value
+
+
+def moe_wq_quantize_weight(fmt, w, groups, K, N, q, scale, stream=None) -> int:
+    return lib().moe_wq_quantize_weight(fmt, ptr(w), groups, K, N, ptr(q), ptr(scale), stream_handle(stream))
+
+
+def moe_wq_workspace_bytes(p: MoeWqParams) -> int:
+    return lib().moe_wq_workspace_bytes(ctypes.byref(p))
+
+
+def moe_block_forward_wq(p: MoeWqParams, stream=None) -> int:
+    return lib().moe_block_forward_wq(ctypes.byref(p), stream_handle(stream))
+
+
 # ------------------------------------------------------------ dense GeGLU FFN
 
 E4B_EMBED_DIM = 2560

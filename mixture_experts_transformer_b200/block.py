@@ -222,6 +222,85 @@ def calibrate(dw: DeviceWeights, x: torch.Tensor, top_k: int = B.TOP_K, router_b
     return tuple(np.float32(v) for v in g), amax.cpu().numpy().astype(np.float32)
 
 
+# ------------------------------------------------ weight-only SFP8 / Q4_0
+
+
+@dataclasses.dataclass
+class WqLinear:
+    """G stacked [K, N] Linears in a weight-only format: the library's blocks
+    (uint8) and, for SFP8, the fp32 matrix scales [G]."""
+
+    q: torch.Tensor
+    scale: torch.Tensor | None
+
+    def struct(self) -> B.MoeWqLinear:
+        return B.MoeWqLinear(B.ptr(self.q), B.ptr(self.scale))
+
+
+@dataclasses.dataclass
+class WqWeights:
+    dims: Dims
+    fmt: str
+    w_router: torch.Tensor
+    wg: WqLinear
+    wu: WqLinear
+    wd: WqLinear
+    sg: WqLinear
+    su: WqLinear
+    sd: WqLinear
+
+
+def quantize_wq_linear(w: torch.Tensor, fmt: str, stream=None) -> WqLinear:
+    """w [G, K, N] or [K, N] bf16 (device) -> the library's format `fmt`."""
+    w3 = w if w.dim() == 3 else w.unsqueeze(0)
+    G, K, N = w3.shape
+    code = B.WFORMATS[fmt]
+    q = torch.empty(B.moe_wq_weight_bytes(code, G, K, N), dtype=torch.uint8, device=w.device)
+    scale = torch.empty(G, dtype=torch.float32, device=w.device) if fmt == "sfp8" else None
+    B.check(B.moe_wq_quantize_weight(code, w3, G, K, N, q, scale, stream), "moe_wq_quantize_weight")
+    return WqLinear(q, scale)
+
+
+def quantize_wq(dw: DeviceWeights, fmt: str, stream=None) -> WqWeights:
+    return WqWeights(dw.dims, fmt, dw.w_router,
+                     *(quantize_wq_linear(t, fmt, stream) for t in (dw.wg, dw.wu, dw.wd, dw.sg, dw.su, dw.sd)))
+
+
+def wq_params(ww: WqWeights, T: int, x, out, *, top_k=B.TOP_K, router_bias=None, res=None,
+              workspace=None) -> B.MoeWqParams:
+    p = B.MoeWqParams()
+    p.T, p.top_k_experts, p.format = T, top_k, B.WFORMATS[ww.fmt]
+    d = ww.dims
+    p.embed_dim, p.num_experts, p.expert_dim, p.hidden_dim = d.embed_dim, d.num_experts, d.expert_dim, d.hidden_dim
+    p.x, p.w_router, p.router_bias = B.ptr(x), B.ptr(ww.w_router), B.ptr(router_bias)
+    for name in ("wg", "wu", "wd", "sg", "su", "sd"):
+        setattr(p, name, getattr(ww, name).struct())
+    p.out = B.ptr(out)
+    if res is not None:
+        p.out_f32, p.idx_out, p.w_out, p.cnt_out = (B.ptr(res.out_f32), B.ptr(res.idx), B.ptr(res.w), B.ptr(res.cnt))
+    if workspace is not None:
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel()
+    return p
+
+
+def forward_wq(ww: WqWeights, x: torch.Tensor, *, top_k: int = B.TOP_K, router_bias=None, debug: bool = False,
+               workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> BlockResult:
+    """One block with weight-only SFP8 / Q4_0 expert and shared Linears."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, ww.dims.embed_dim), dtype=torch.bfloat16, device=x.device)
+    res = BlockResult(out=out)
+    if debug:
+        res.out_f32 = torch.empty((T, ww.dims.embed_dim), dtype=torch.float32, device=x.device)
+        res.idx = torch.empty((T, top_k), dtype=torch.int32, device=x.device)
+        res.w = torch.empty((T, top_k), dtype=torch.float32, device=x.device)
+        res.cnt = torch.empty((ww.dims.num_experts,), dtype=torch.int32, device=x.device)
+    p = wq_params(ww, T, x, out, top_k=top_k, router_bias=router_bias, res=res, workspace=workspace)
+    B.check(B.moe_block_forward_wq(p, stream), "moe_block_forward_wq")
+    return res
+
+
 # ---------------------------------------------------------------- dense FFN
 
 

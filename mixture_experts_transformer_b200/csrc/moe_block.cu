@@ -18,6 +18,7 @@
 #include "permute.cuh"
 #include "router.cuh"
 #include "nvfp4.cuh"
+#include "wq_gemm.cuh"
 
 namespace moe {
 
@@ -195,6 +196,15 @@ moe_status device_state(DeviceState** out) {
       }
       if (cudaFuncSetAttribute(fp4_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
           cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (cudaFuncSetAttribute(wq_gemm_kernel<kWfSfp8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kWqSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(wq_gemm_kernel<kWfSfp8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kWqSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(wq_gemm_kernel<kWfQ4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kWqSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(wq_gemm_kernel<kWfQ4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kWqSmemBytes) != cudaSuccess)
         return MOE_ERR_CUDA;
       if (cudaFuncSetAttribute(fp4_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF4SmemBytes) !=
           cudaSuccess)
@@ -466,20 +476,23 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
 }
 
 // Scan of the bitmasks, then the scatter (and, with x, the copy into x_perm).
+// allow_pairs = false: tiles of one 128-row block only (the weight-only GEMMs).
 moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const int32_t* idx, const void* x,
-                           int32_t* cnt, int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st) {
+                           int32_t* cnt, int32_t* off, int32_t* row_of, int32_t* token_of, cudaStream_t st,
+                           bool allow_pairs = true) {
   const uint32_t* masks = reinterpret_cast<const uint32_t*>(ws + L.masks);
   int32_t* base = reinterpret_cast<int32_t*>(ws + L.base);
   DeviceState* s = nullptr;
   MOE_TRY(device_state(&s));
-  const bool pairs = pair_sm(d, s);
+  const bool pairs = allow_pairs && pair_sm(d, s);
   {
     LaunchScope ls_(kKRouteScan, st);
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
                                      reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256,
-                                     paired_gateup(d) ? 1 : 0, (pairs || paired_down(d)) ? 1 : 0, d.e0, d.el);
+                                     (allow_pairs && paired_gateup(d)) ? 1 : 0,
+                                     (pairs || (allow_pairs && paired_down(d))) ? 1 : 0, d.e0, d.el);
     MOE_TRY(ls_.done(le_));
   }
   const long long R = static_cast<long long>(d.T) * d.k;
@@ -812,6 +825,123 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     MOE_TRY(ls_.done(le_));
   }
   const size_t R = static_cast<size_t>(d.T) * d.k;
+  if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->w_out && cudaMemcpyAsync(p->w_out, w, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (p->cnt_out && cudaMemcpyAsync(p->cnt_out, cnt, d.E * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+// -------------------------------------------------- weight-only formats
+
+size_t wq_bytes(int fmt, size_t groups, size_t K, size_t N) {
+  const size_t blk = fmt == MOE_WFMT_SFP8 ? wq_block_bytes<kWfSfp8>() : wq_block_bytes<kWfQ4>();
+  return groups * ((N + 127) / 128) * (K / kBK) * blk;
+}
+
+bool wq_linear_ok(int fmt, const moe_wq_linear& l) {
+  return l.q && aligned16(l.q) && (fmt != MOE_WFMT_SFP8 || (l.scale && aligned4(l.scale)));
+}
+
+moe_status check_wq_args(const moe_wq_params* p, Dims* d) {
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (p->format != MOE_WFMT_SFP8 && p->format != MOE_WFMT_Q4_0) return MOE_ERR_INVALID_ARG;
+  d->T = p->T;
+  d->k = p->top_k_experts;
+  d->D = p->embed_dim ? p->embed_dim : MOE_EMBED_DIM;
+  d->E = p->num_experts ? p->num_experts : MOE_NUM_EXPERTS;
+  d->F = p->expert_dim ? p->expert_dim : MOE_EXPERT_DIM;
+  d->S = p->hidden_dim ? p->hidden_dim : MOE_HIDDEN_DIM;
+  d->e0 = 0;
+  d->el = d->E;
+  if (!dims_ok(*d)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  if (!p->x || !p->w_router || !p->out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(p->x) || !aligned16(p->w_router) || !aligned16(p->out)) return MOE_ERR_ALIGNMENT;
+  const moe_wq_linear* ls[] = {&p->wg, &p->wu, &p->wd, &p->sg, &p->su, &p->sd};
+  for (const moe_wq_linear* l : ls)
+    if (!wq_linear_ok(p->format, *l)) return (l->q && (p->format != MOE_WFMT_SFP8 || l->scale)) ? MOE_ERR_ALIGNMENT
+                                                                                                 : MOE_ERR_INVALID_ARG;
+  if (p->out_f32 && !aligned16(p->out_f32)) return MOE_ERR_ALIGNMENT;
+  const void* opt4[] = {p->router_bias, p->idx_out, p->w_out, p->cnt_out};
+  for (const void* q : opt4)
+    if (q && !aligned4(q)) return MOE_ERR_ALIGNMENT;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(p->x), ob = reinterpret_cast<uintptr_t>(p->out);
+  const uintptr_t bytes = static_cast<uintptr_t>(d->T) * d->D * 2;
+  if (xb < ob + bytes && ob < xb + bytes) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+template <int FMT, bool GATEUP>
+cudaError_t launch_wq(int grid, cudaStream_t st, const WqParams& P) {
+  return launch_k(wq_gemm_kernel<FMT, GATEUP>, grid, kWqThreads, kWqSmemBytes, st, P);
+}
+
+moe_status enqueue_block_wq(const moe_wq_params* p, const Dims& d, const Layout& L, uint8_t* ws, DeviceState* s,
+                            cudaStream_t st) {
+  const size_t R = static_cast<size_t>(d.T) * d.k;
+  int32_t* idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  float* w = reinterpret_cast<float*>(ws + L.w);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  int32_t* off = reinterpret_cast<int32_t*>(ws + L.off);
+  int32_t* row_of = reinterpret_cast<int32_t*>(ws + L.row_of);
+  int32_t* token_of = reinterpret_cast<int32_t*>(ws + L.token_of);
+  __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+  __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + L.y);
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(ws + L.hs);
+  float* sbuf = reinterpret_cast<float*>(ws + L.s);
+  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
+  TileCounts* counts = reinterpret_cast<TileCounts*>(ws + L.counts);
+  const bool sfp = p->format == MOE_WFMT_SFP8;
+
+  MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
+  MOE_TRY(enqueue_permute(d, L, ws, idx, p->x, cnt, off, row_of, token_of, st, false));
+
+  auto sc = [&](const moe_wq_linear& l) { return sfp ? l.scale : static_cast<const float*>(nullptr); };
+  WqParams gu;
+  std::memset(&gu, 0, sizeof(gu));
+  if (!map_2d(&gu.tmA[0], x_perm, R, d.D, kBM) || !map_2d(&gu.tmA[1], p->x, d.T, d.D, kBM) ||
+      !map_2d(&gu.tmAs[0], x_perm, R, d.D, kASmallRows) || !map_2d(&gu.tmAs[1], p->x, d.T, d.D, kASmallRows))
+    return MOE_ERR_CUDA;
+  gu.prob[0] = WqProblem{d.D, d.F, d.E, static_cast<int>(R), p->wg.q, p->wu.q, sc(p->wg), sc(p->wu), h, d.F, 0};
+  gu.prob[1] = WqProblem{d.D, d.S, 1, d.T, p->sg.q, p->su.q, sc(p->sg), sc(p->su), hs, d.S, 0};
+  gu.nprob = 2;
+  gu.a_small = 1;
+  gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
+  gu.num_tiles = &counts->gateup;
+  gu.next_tile = &counts->next_gateup;
+  gu.err = s->err;
+  {
+    LaunchScope ls_(kKGemmGateUp, st);
+    const int grid = std::min(s->sm_count, L.max_tiles_gu);
+    MOE_TRY(ls_.done(sfp ? launch_wq<kWfSfp8, true>(grid, st, gu) : launch_wq<kWfQ4, true>(grid, st, gu)));
+  }
+  WqParams dn;
+  std::memset(&dn, 0, sizeof(dn));
+  if (!map_2d(&dn.tmA[0], h, R, d.F, kBM) || !map_2d(&dn.tmA[1], hs, d.T, d.S, kBM) ||
+      !map_2d(&dn.tmAs[0], h, R, d.F, kASmallRows) || !map_2d(&dn.tmAs[1], hs, d.T, d.S, kASmallRows))
+    return MOE_ERR_CUDA;
+  dn.prob[0] = WqProblem{d.F, d.D, d.E, static_cast<int>(R), p->wd.q, nullptr, sc(p->wd), nullptr, y, d.D, 0};
+  dn.prob[1] = WqProblem{d.S, d.D, 1, d.T, p->sd.q, nullptr, sc(p->sd), nullptr, sbuf, d.D, 1};
+  dn.nprob = 2;
+  dn.a_small = 1;
+  dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
+  dn.num_tiles = &counts->down;
+  dn.next_tile = &counts->next_down;
+  dn.err = s->err;
+  {
+    LaunchScope ls_(kKGemmDown, st);
+    const int grid = std::min(s->sm_count, L.max_tiles_dn);
+    MOE_TRY(ls_.done(sfp ? launch_wq<kWfSfp8, false>(grid, st, dn) : launch_wq<kWfQ4, false>(grid, st, dn)));
+  }
+  {
+    LaunchScope ls_(kKCombine, st);
+    const int dsplit = std::max(1, std::min(4, (2 * s->sm_count) / std::max(1, d.T)));
+    MOE_TRY(ls_.done(launch_k(combine_kernel, dim3(d.T, dsplit), 128, 0, st, sbuf, y, row_of, w, d.T, d.k, d.D,
+                              static_cast<int>(R), static_cast<__nv_bfloat16*>(p->out), p->out_f32, s->err)));
+  }
   if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (p->w_out && cudaMemcpyAsync(p->w_out, w, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -1259,6 +1389,85 @@ moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* 
   L.masks = partial_bytes;
   return enqueue_route(d, L, scratch, p->x, p->w_router, p->router_bias, idx, w, static_cast<cudaStream_t>(stream),
                        p->logits_out);
+}
+
+moe_status moe_wq_weight_bytes(int format, int groups, int K, int N, size_t* bytes) {
+  if (format != MOE_WFMT_SFP8 && format != MOE_WFMT_Q4_0) return MOE_ERR_INVALID_ARG;
+  if (groups <= 0 || K <= 0 || N <= 0 || K % 64 || N % 64) return MOE_ERR_INVALID_ARG;
+  if (bytes) *bytes = wq_bytes(format, groups, K, N);
+  return MOE_OK;
+}
+
+moe_status moe_wq_quantize_weight(int format, const void* w, int groups, int K, int N, uint8_t* q, float* scale,
+                                  void* stream) {
+  t_launches = 0;
+  if (format != MOE_WFMT_SFP8 && format != MOE_WFMT_Q4_0) return MOE_ERR_INVALID_ARG;
+  if (groups <= 0 || K <= 0 || N <= 0 || K % 64 || N % 64 || groups > 65535) return MOE_ERR_INVALID_ARG;
+  const bool sfp = format == MOE_WFMT_SFP8;
+  if (!w || !q || (sfp && !scale)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(q) || (sfp && !aligned4(scale))) return MOE_ERR_ALIGNMENT;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(q, 0, wq_bytes(format, groups, K, N), st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (sfp) {
+    if (cudaMemsetAsync(scale, 0, sizeof(float) * groups, st) != cudaSuccess) return MOE_ERR_CUDA;
+    const size_t per_group = static_cast<size_t>(K) * N;
+    uint32_t* amax_bits = reinterpret_cast<uint32_t*>(scale);  // amax first, then the scale in place
+    {
+      const int bpg = static_cast<int>(std::min<size_t>((per_group / 8 + 255) / 256, 64));
+      LaunchScope ls_(kKWeightAmax, st);
+      MOE_TRY(ls_.done(launch_k(weight_amax_kernel, dim3(bpg, groups), 256, 0, st,
+                                static_cast<const __nv_bfloat16*>(w), per_group, amax_bits)));
+    }
+    LaunchScope ls_(kKTensorScale, st);
+    MOE_TRY(ls_.done(launch_k(sfp8_scale_kernel, (groups + 127) / 128, 128, 0, st,
+                              static_cast<const uint32_t*>(amax_bits), scale, groups)));
+  }
+  const long long items = static_cast<long long>(N) * (K / 64);
+  const dim3 grid(static_cast<unsigned>((items + 127) / 128), groups);
+  LaunchScope ls_(kKWeightQuant, st);
+  return ls_.done(sfp ? launch_k(wq_quant_kernel<kWfSfp8>, grid, 128, 0, st, static_cast<const __nv_bfloat16*>(w), K,
+                                 N, static_cast<const float*>(scale), q)
+                      : launch_k(wq_quant_kernel<kWfQ4>, grid, 128, 0, st, static_cast<const __nv_bfloat16*>(w), K,
+                                 N, static_cast<const float*>(nullptr), q));
+}
+
+size_t moe_wq_workspace_bytes(const moe_wq_params* p) {
+  if (!p) return 0;
+  Dims d;
+  d.T = p->T;
+  d.k = p->top_k_experts;
+  d.D = p->embed_dim ? p->embed_dim : MOE_EMBED_DIM;
+  d.E = p->num_experts ? p->num_experts : MOE_NUM_EXPERTS;
+  d.F = p->expert_dim ? p->expert_dim : MOE_EXPERT_DIM;
+  d.S = p->hidden_dim ? p->hidden_dim : MOE_HIDDEN_DIM;
+  d.e0 = 0;
+  d.el = d.E;
+  if (!dims_ok(d)) return 0;
+  return make_layout(d).total;
+}
+
+moe_status moe_block_forward_wq(const moe_wq_params* p, void* stream) {
+  t_launches = 0;
+  Dims d;
+  MOE_TRY(check_wq_args(p, &d));
+  if (d.T == 0) return MOE_OK;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  const Layout L = make_layout(d);
+  uint8_t* ws = nullptr;
+  if (p->workspace) {
+    if ((reinterpret_cast<uintptr_t>(p->workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGNMENT;
+    if (p->workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    ws = static_cast<uint8_t*>(p->workspace);
+  } else {
+    void* wsv = nullptr;
+    MOE_TRY(library_workspace(s, L.total, &wsv));
+    ws = static_cast<uint8_t*>(wsv);
+  }
+  return enqueue_block_wq(p, d, L, ws, s, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_nvfp4_weight_bytes(int groups, int K, int N, size_t* q_bytes, size_t* sf_bytes) {

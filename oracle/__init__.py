@@ -12,6 +12,9 @@ to be read against the pages:
 * ``moe_oracle`` - router, softmax, top-k, renormalisation, permutation,
   GeGLU experts, shared MLP, branch sum, inter-block RMSNorm;
 * ``nvfp4``     - e2m1 / e4m3 codecs and the group-16 NVFP4 quantiser;
+* ``wformats``  - the weight-only formats SFP8 and Q4_0 (readings stated in
+  the module) and the block on weights in those formats;
+* ``sandwich``  - the pre/post-FFN RMSNorm sandwich and residual;
 * ``counts``    - parameter counts implied by the layer shapes.
 
 Parity status: every function is pinned by a ``-m "not gpu"`` test to

@@ -145,9 +145,12 @@ def moe_block_wq(x, w_router, wg, wu, wd, sg, su, sd, fmt: str, top_k: int = 8, 
     def deq(m):
         return weight_fake_quantize(mo.f64(m).astype(np.float32), fmt)
 
-    e_count = wg.shape[0]
-    wgq = np.stack([deq(wg[e]) for e in range(e_count)])
-    wuq = np.stack([deq(wu[e]) for e in range(e_count)])
-    wdq = np.stack([deq(wd[e]) for e in range(e_count)])
+    if routing is None:
+        idx, w, _ = mo.route(x, w_router, top_k, bias)
+        routing = (idx, w)
+    # only the experts the routing uses are quantised; the others stay zero
+    wgq, wuq, wdq = (np.zeros(a.shape) for a in (wg, wu, wd))
+    for e in np.unique(np.asarray(routing[0])):
+        wgq[e], wuq[e], wdq[e] = deq(wg[e]), deq(wu[e]), deq(wd[e])
     return mo.moe_block(x, w_router, wgq, wuq, wdq, deq(sg), deq(su), deq(sd), top_k=top_k, bias=bias,
                         routing=routing)
