@@ -57,7 +57,8 @@ typedef enum {
   MOE_ERR_ARCH = 3,          /* the current device is not sm_100 */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, allocation) */
   MOE_ERR_WORKSPACE = 5,     /* caller workspace smaller than moe_workspace_bytes_ex */
-  MOE_ERR_DEVICE_TIMEOUT = 6 /* a kernel's bounded wait ran out (reported by moe_get_device_status) */
+  MOE_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out (reported by moe_get_device_status) */
+  MOE_ERR_GUARD = 7           /* a workspace guard word was overwritten (reported by moe_get_device_status) */
 } moe_status;
 
 /* Gemma-4-26B-A4B block constants (TransformerConfig of gm.nn.Gemma4_26B_A4B). */
@@ -122,6 +123,14 @@ typedef enum {
  * a reduce-scatter) and rounds with moe_round_bf16. A shard may not use
  * norm_post or residual, which act on the full sum.
  * out may be NULL when out_f32 is given: only the fp32 result is written.
+ *
+ * Debug aid: with check_guards nonzero, the block writes a pattern into the
+ * 256 guard bytes that end every workspace layout (moe_ws_layout.guard)
+ * before its first kernel and checks it after its last (two extra launches);
+ * a kernel that wrote past the workspace's data then shows as MOE_ERR_GUARD
+ * from moe_get_device_status. The block's kernels also range-check every
+ * index they read back from the workspace and record MOE_ERR_INVALID_ARG
+ * instead of addressing memory out of range.
  */
 typedef struct moe_params {
   int T;
@@ -152,6 +161,7 @@ typedef struct moe_params {
   float* logits_out;
   int expert_begin;
   int expert_count;
+  int check_guards;
 } moe_params;
 
 /*
@@ -173,6 +183,7 @@ typedef struct moe_ws_layout {
   size_t x_perm, h, y, hs, s;
   size_t idx, w, cnt, off, row_of, token_of;
   size_t x_norm;
+  size_t guard;  /* 256 guard bytes, the last of the layout */
 } moe_ws_layout;
 
 /* Bytes of workspace a call with these params needs (T, top_k and dims are read). */
@@ -520,6 +531,13 @@ moe_status moe_dense_ffn_forward(const moe_dense_params* p, void* stream);
  * summed across expert shards.
  */
 moe_status moe_round_bf16(const float* in, void* out, size_t n, void* stream);
+
+/*
+ * Check the guard words of the caller workspace p->workspace (laid out for
+ * p's dims) on their own: MOE_ERR_GUARD from the next moe_get_device_status
+ * if they differ from the pattern a guarded call wrote.
+ */
+moe_status moe_workspace_guard_check(const moe_params* p, void* stream);
 
 /* Human-readable name of a status code. */
 const char* moe_status_string(moe_status s);

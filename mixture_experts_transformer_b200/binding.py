@@ -20,6 +20,7 @@ MOE_ERR_ARCH = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_WORKSPACE = 5
 MOE_ERR_DEVICE_TIMEOUT = 6
+MOE_ERR_GUARD = 7
 
 EMBED_DIM, NUM_EXPERTS, EXPERT_DIM, HIDDEN_DIM, TOP_K = 2816, 128, 704, 2112, 8
 
@@ -56,6 +57,7 @@ class MoeParams(ctypes.Structure):
         ("logits_out", _vp),
         ("expert_begin", ctypes.c_int),
         ("expert_count", ctypes.c_int),
+        ("check_guards", ctypes.c_int),
     ]
 
 
@@ -63,7 +65,7 @@ class MoeWsLayout(ctypes.Structure):
     _fields_ = [
         (name, ctypes.c_size_t)
         for name in ("total_bytes", "x_perm", "h", "y", "hs", "s", "idx", "w", "cnt", "off", "row_of", "token_of",
-                     "x_norm")
+                     "x_norm", "guard")
     ]
 
 
@@ -80,6 +82,7 @@ EXPORTS = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_launch_count": (ctypes.c_int, []),
     "moe_round_bf16": (ctypes.c_int, [_vp, _vp, ctypes.c_size_t, _vp]),
+    "moe_workspace_guard_check": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp]),
     "moe_block_forward_hostio": (ctypes.c_int, [ctypes.POINTER(MoeParams), _vp, _vp, _vp]),
     "moe_profile_begin": (ctypes.c_int, [ctypes.c_uint32]),
     "moe_profile_end": (ctypes.c_int, [_vp, _vp, ctypes.c_int]),
@@ -164,6 +167,7 @@ def make_params(
     logits_out=None,
     expert_begin: int = 0,
     expert_count: int = 0,
+    check_guards: bool = False,
 ) -> MoeParams:
     p = MoeParams()
     p.T = T
@@ -198,6 +202,7 @@ def make_params(
         setattr(p, name, ptr(val))
     p.residual = 1 if residual else 0
     p.expert_begin, p.expert_count = expert_begin, expert_count
+    p.check_guards = 1 if check_guards else 0
     if workspace is not None and not workspace_bytes:
         workspace_bytes = workspace.numel() * workspace.element_size()
     p.workspace_bytes = workspace_bytes
@@ -252,6 +257,10 @@ def moe_status_string(status: int) -> str:
 
 def moe_last_launch_count() -> int:
     return lib().moe_last_launch_count()
+
+
+def moe_workspace_guard_check(p: MoeParams, stream=None) -> int:
+    return lib().moe_workspace_guard_check(ctypes.byref(p), stream_handle(stream))
 
 
 def moe_round_bf16(src, dst, n: int, stream=None) -> int:

@@ -4,6 +4,7 @@
 // down GEMM -> combine, all on the caller's stream with no host sync.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstdint>
@@ -43,6 +44,7 @@ struct Layout {
   size_t total;
   size_t partial, idx, w, masks, base, cnt, off, row_of, token_of, tiles_gu, tiles_dn, counts;
   size_t x_perm, h, y, hs, s, x_norm;
+  size_t guard;  // 256 bytes of guard words after the data (written and checked only on request)
   int nsplit, nchunks, max_tiles_gu, max_tiles_dn;
 };
 
@@ -103,6 +105,7 @@ Layout make_layout(const Dims& d) {
   L.hs = take(T * d.S * 2);
   L.s = take(T * d.D * 4);
   L.x_norm = take(T * d.D * 2);
+  L.guard = take(kGuardWords * 4);
   L.total = o;
   return L;
 }
@@ -325,6 +328,7 @@ enum KernelId : int {
   kKCombineNorm,
   kKAmax,
   kKPreNorm,
+  kKGuard,
   kKCount
 };
 const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "build_masks", "route_scan",
@@ -332,7 +336,8 @@ const char* const kKernelNames[kKCount] = {"router_logits", "router_topk", "buil
                                            "grouped_gemm_down", "combine", "timeout_probe",
                                            "nvfp4_weight_amax", "nvfp4_tensor_scale", "nvfp4_weight_quant",
                                            "nvfp4_act_quant", "route_scatter_fp4", "fp4_gemm_gateup",
-                                           "fp4_gemm_down", "combine_norm", "amax", "rms_norm_pre"};
+                                           "fp4_gemm_down", "combine_norm", "amax", "rms_norm_pre",
+                                           "workspace_guard"};
 
 struct ProfRecord {
   int id;
@@ -355,16 +360,22 @@ cudaEvent_t pooled_event() {
 }
 
 // Brackets one kernel launch with timing events when profiling is on.
+// Also an NVTX range named after the kernel around its launch (a profiler's
+// timeline shows which library kernel each launch is; no cost without one).
 struct LaunchScope {
   cudaStream_t st;
   int id;
   cudaEvent_t a = nullptr;
   LaunchScope(int id_, cudaStream_t st_) : st(st_), id(id_) {
+    nvtxRangePushA(kKernelNames[id]);
     if (t_profiling && ((t_profile_mask >> id) & 1u)) {
       a = pooled_event();
       cudaEventRecord(a, st);
     }
   }
+  ~LaunchScope() { nvtxRangePop(); }
+  LaunchScope(const LaunchScope&) = delete;
+  LaunchScope& operator=(const LaunchScope&) = delete;
   moe_status done(cudaError_t launch_err) {
     ++t_launches;
     if (t_profiling && a) {
@@ -394,6 +405,14 @@ cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
+
+// An NVTX range around a public entry point.
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+  ApiRange(const ApiRange&) = delete;
+  ApiRange& operator=(const ApiRange&) = delete;
+};
 
 #define MOE_TRY(expr)                   \
   do {                                  \
@@ -520,6 +539,11 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm);
   TileCounts* counts = reinterpret_cast<TileCounts*>(ws + L.counts);
 
+  uint32_t* guard = reinterpret_cast<uint32_t*>(ws + L.guard);
+  if (p->check_guards) {
+    LaunchScope ls_(kKGuard, st);
+    MOE_TRY(ls_.done(launch_k(guard_fill_kernel, 1, kGuardWords, 0, st, guard)));
+  }
   // the block's input: x, or its pre-FFN RMSNorm (bf16, in the workspace)
   const void* xin = p->x;
   if (p->norm_pre) {
@@ -610,6 +634,10 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   MOE_TRY(ls_.done(le_));
   }
 
+  if (p->check_guards) {
+    LaunchScope ls_(kKGuard, st);
+    MOE_TRY(ls_.done(launch_k(guard_check_kernel, 1, kGuardWords, 0, st, static_cast<const uint32_t*>(guard), s->err)));
+  }
   if (p->idx_out && cudaMemcpyAsync(p->idx_out, idx, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (p->w_out && cudaMemcpyAsync(p->w_out, w, R * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
@@ -1166,10 +1194,12 @@ moe_status moe_workspace_layout(const moe_params* p, moe_ws_layout* out) {
   out->row_of = L.row_of;
   out->token_of = L.token_of;
   out->x_norm = L.x_norm;
+  out->guard = L.guard;
   return MOE_OK;
 }
 
 moe_status moe_block_forward_ex(const moe_params* p, void* stream) {
+  ApiRange nvtx_range_("moe_block_forward_ex");
   t_launches = 0;
   Dims d;
   MOE_TRY(check_block_args(p, &d));
@@ -1202,6 +1232,7 @@ moe_status moe_block_forward(const void* x, const void* w_router, const void* wg
 }
 
 moe_status moe_route(const moe_params* p, int32_t* idx, float* w, void* stream) {
+  ApiRange nvtx_range_("moe_route");
   t_launches = 0;
   if (!p) return MOE_ERR_INVALID_ARG;
   const Dims d = dims_of(p);
@@ -1223,6 +1254,7 @@ moe_status moe_route(const moe_params* p, int32_t* idx, float* w, void* stream) 
 
 moe_status moe_permute(const moe_params* p, const int32_t* idx, int32_t* cnt, int32_t* off, int32_t* row_of,
                        int32_t* token_of, void* stream) {
+  ApiRange nvtx_range_("moe_permute");
   t_launches = 0;
   if (!p) return MOE_ERR_INVALID_ARG;
   const Dims d = dims_of(p);
@@ -1258,7 +1290,8 @@ moe_status moe_get_device_status(void* stream) {
   if (cudaMemcpy(&word, s->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (word) {
     if (cudaMemset(s->err, 0, sizeof(word)) != cudaSuccess) return MOE_ERR_CUDA;
-    return (word & kErrWaitTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_INVALID_ARG;
+    if (word & kErrWaitTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+    return (word & kErrGuard) ? MOE_ERR_GUARD : MOE_ERR_INVALID_ARG;
   }
   return MOE_OK;
 }
@@ -1285,13 +1318,32 @@ const char* moe_status_string(moe_status st) {
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_GUARD: return "MOE_ERR_GUARD";
   }
   return "MOE_ERR_UNKNOWN";
 }
 
 int moe_last_launch_count(void) { return t_launches; }
 
+moe_status moe_workspace_guard_check(const moe_params* p, void* stream) {
+  t_launches = 0;
+  ApiRange nvtx_range_("moe_workspace_guard_check");
+  if (!p || !p->workspace) return MOE_ERR_INVALID_ARG;
+  const Dims d = dims_of(p);
+  if (!dims_ok(d)) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(d);
+  if ((reinterpret_cast<uintptr_t>(p->workspace) & (kAlign - 1)) != 0) return MOE_ERR_ALIGNMENT;
+  if (p->workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+  DeviceState* s = nullptr;
+  MOE_TRY(device_state(&s));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LaunchScope ls_(kKGuard, st);
+  return ls_.done(launch_k(guard_check_kernel, 1, kGuardWords, 0, st,
+                           reinterpret_cast<const uint32_t*>(static_cast<uint8_t*>(p->workspace) + L.guard), s->err));
+}
+
 moe_status moe_round_bf16(const float* in, void* out, size_t n, void* stream) {
+  ApiRange nvtx_range_("moe_round_bf16");
   t_launches = 0;
   if (n == 0) return MOE_OK;
   if (!in || !out || n % 8) return MOE_ERR_INVALID_ARG;
@@ -1308,6 +1360,7 @@ moe_status moe_round_bf16(const float* in, void* out, size_t n, void* stream) {
 }
 
 moe_status moe_block_forward_hostio(const moe_params* p, const void* x_host, void* out_host, void* stream) {
+  ApiRange nvtx_range_("moe_block_forward_hostio");
   t_launches = 0;
   Dims d;
   MOE_TRY(check_block_args(p, &d));
@@ -1363,6 +1416,7 @@ int moe_profile_end(float* total_ms, int* launches, int n) {
 const char* moe_kernel_name(int id) { return (id >= 0 && id < kKCount) ? kKernelNames[id] : nullptr; }
 
 moe_status moe_route_noalloc(const moe_params* p, int32_t* idx, float* w, void* stream) {
+  ApiRange nvtx_range_("moe_route_noalloc");
   t_launches = 0;
   if (!p) return MOE_ERR_INVALID_ARG;
   const Dims d = dims_of(p);
@@ -1400,6 +1454,7 @@ moe_status moe_wq_weight_bytes(int format, int groups, int K, int N, size_t* byt
 
 moe_status moe_wq_quantize_weight(int format, const void* w, int groups, int K, int N, uint8_t* q, float* scale,
                                   void* stream) {
+  ApiRange nvtx_range_("moe_wq_quantize_weight");
   t_launches = 0;
   if (format != MOE_WFMT_SFP8 && format != MOE_WFMT_Q4_0) return MOE_ERR_INVALID_ARG;
   if (groups <= 0 || K <= 0 || N <= 0 || K % 64 || N % 64 || groups > 65535) return MOE_ERR_INVALID_ARG;
@@ -1449,6 +1504,7 @@ size_t moe_wq_workspace_bytes(const moe_wq_params* p) {
 }
 
 moe_status moe_block_forward_wq(const moe_wq_params* p, void* stream) {
+  ApiRange nvtx_range_("moe_block_forward_wq");
   t_launches = 0;
   Dims d;
   MOE_TRY(check_wq_args(p, &d));
@@ -1479,6 +1535,7 @@ moe_status moe_nvfp4_weight_bytes(int groups, int K, int N, size_t* q_bytes, siz
 
 moe_status moe_nvfp4_quantize_weight(const void* w, int groups, int K, int N, uint8_t* q, uint8_t* sf, float* g,
                                      void* stream) {
+  ApiRange nvtx_range_("moe_nvfp4_quantize_weight");
   t_launches = 0;
   if (groups <= 0 || K <= 0 || N <= 0 || K % 64 || N % 64 || groups > 65535) return MOE_ERR_INVALID_ARG;
   if (!w || !q || !sf || !g) return MOE_ERR_INVALID_ARG;
@@ -1511,6 +1568,7 @@ moe_status moe_nvfp4_quantize_weight(const void* w, int groups, int K, int N, ui
 }
 
 moe_status moe_nvfp4_quantize_act(const void* x, int rows, int K, float g, uint8_t* q, uint8_t* sf, void* stream) {
+  ApiRange nvtx_range_("moe_nvfp4_quantize_act");
   t_launches = 0;
   if (rows < 0 || K <= 0 || K % 64 || !(g > 0.f)) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
@@ -1560,6 +1618,7 @@ moe_status moe_nvfp4_workspace_layout(const moe_nvfp4_params* p, moe_nvfp4_ws_la
 }
 
 moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream) {
+  ApiRange nvtx_range_("moe_block_forward_nvfp4");
   t_launches = 0;
   Dims d;
   MOE_TRY(check_fp4_args(p, &d));
@@ -1582,6 +1641,7 @@ moe_status moe_block_forward_nvfp4(const moe_nvfp4_params* p, void* stream) {
 }
 
 moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, float* scales, void* stream) {
+  ApiRange nvtx_range_("moe_nvfp4_calibrate");
   t_launches = 0;
   Dims d;
   MOE_TRY(check_block_args(p, &d));
@@ -1624,6 +1684,7 @@ size_t moe_dense_workspace_bytes(const moe_dense_params* p) {
 }
 
 moe_status moe_dense_ffn_forward(const moe_dense_params* p, void* stream) {
+  ApiRange nvtx_range_("moe_dense_ffn_forward");
   t_launches = 0;
   if (!p) return MOE_ERR_INVALID_ARG;
   const DenseDims d = dense_dims(p);

@@ -402,6 +402,23 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
   }
 }
 
+// Workspace guard words (a debug aid): the pattern a guarded call writes
+// after its workspace data before its first kernel, and the check after its
+// last kernel, which records kErrGuard when any word changed.
+constexpr uint32_t kGuardPattern = 0x5AC3E13Bu;
+constexpr int kGuardWords = 64;  // 256 bytes
+
+__global__ void guard_fill_kernel(uint32_t* __restrict__ g) {
+  pdl_wait_then_release();
+  if (threadIdx.x < kGuardWords) g[threadIdx.x] = kGuardPattern ^ (threadIdx.x * 0x9E3779B9u);
+}
+
+__global__ void guard_check_kernel(const uint32_t* __restrict__ g, uint32_t* __restrict__ err) {
+  pdl_wait_then_release();
+  if (threadIdx.x < kGuardWords && g[threadIdx.x] != (kGuardPattern ^ (threadIdx.x * 0x9E3779B9u)))
+    atomicOr(err, kErrGuard);
+}
+
 // A kernel that waits, bounded, on a barrier nothing completes: the failure
 // path of every bounded wait in the library, exercised on purpose.
 __global__ void timeout_probe_kernel(uint32_t* err, unsigned long long timeout_ns) {

@@ -16,6 +16,7 @@ enum : uint32_t {
   kErrWaitTimeout = 1u,  // a bounded mbarrier / flag wait ran out
   kErrBadTile = 2u,      // a work-list entry failed its range check
   kErrBadIndex = 4u,     // an expert index outside [0, num_experts), or a routed row outside its buffer
+  kErrGuard = 8u,        // a workspace guard word was overwritten
 };
 
 // Nanoseconds a kernel waits on one barrier phase before it gives up.

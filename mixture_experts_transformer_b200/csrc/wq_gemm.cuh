@@ -29,17 +29,22 @@
 //
 // Roles (512 threads, one CTA per SM; 16 warps, so 4 per SM sub-partition):
 //   warp 0        producer: tiles from the work counter into the tile ring,
-//                 and copy thread 0 of every stage
+//                 and the A rows of every stage into the A ring
 //   warp 1        MMA issuer: waits for a stage's A rows and decoded weights,
 //                 4 x tcgen05.mma (K = 16), frees both
 //   warps 2..5    epilogue, one per TMEM lane quarter
 //   warps 6..13   converters: a stage's codes -> bf16 weights (K-major, 128-byte
 //                 swizzle) in a 2-deep ring, then a proxy fence and arrival
-//   warps 14, 15  copy threads 1, 2 (one thread issues ~2.2 M copies per
-//                 second; a stage's copies - the A rows and two weight blocks -
-//                 go to different threads)
-// Shared memory: 4 stages x (16 KB A + 16 KB codes), 2 x 32 KB decoded
-// weights. TMEM: 2 accumulators x 256 columns.
+//   warps 14, 15  the weight blocks of every stage (block 0 and block 1) into
+//                 the code ring (one thread issues ~2.2 M copies per second,
+//                 so the A copy and the two block copies go to three threads)
+// The rings are separate: A slots are freed by the MMAs, code slots by the
+// converters as soon as they have read them. The weight stream, which carries
+// nearly all of the bytes at small batches, so runs as far ahead as the code
+// ring is deep (5 stages of SFP8, 8 of Q4_0), not only as far as the
+// converters may run ahead of the MMAs.
+// Shared memory: A ring 4 x 16 KB, code ring 80 KB, decoded weights 2 x 32 KB.
+// TMEM: 2 accumulators x 256 columns.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -56,18 +61,27 @@ __host__ __device__ constexpr int wq_block_bytes() {
   return FMT == kWfSfp8 ? 8192 : 4608;
 }
 
-constexpr int kWqStages = 4;
+constexpr int kWqAStages = 4;
 constexpr int kWqBStages = 2;
 constexpr int kWqEpiWarps = 4;
 constexpr int kWqConvWarps = 8;
-constexpr int kWqCopyWarps = 2;
-constexpr int kWqNProd = 1 + kWqCopyWarps;
+constexpr int kWqCopyWarps = 2;  // the two weight-block issuers
 constexpr int kWqThreads = 32 * (2 + kWqEpiWarps + kWqConvWarps + kWqCopyWarps);
 constexpr int kWqConvThreads = 32 * kWqConvWarps;
-constexpr int kWqCodeStage = 2 * 8192;          // two 128-row weight blocks per stage
+constexpr int kWqCodeRing = 80 * 1024;          // code ring bytes
+constexpr int kWqMaxCStages = 8;
+template <int FMT>
+__host__ __device__ constexpr int wq_code_stage() {  // two 128-row weight blocks
+  return 2 * wq_block_bytes<FMT>();
+}
+template <int FMT>
+__host__ __device__ constexpr int wq_cstages() {
+  return kWqCodeRing / wq_code_stage<FMT>() < kWqMaxCStages ? kWqCodeRing / wq_code_stage<FMT>() : kWqMaxCStages;
+}
 constexpr int kWqBStage = 256 * kBK * 2;        // 256 weight rows x 64 K bf16
-constexpr int kWqSmemBytes = kWqStages * (kAStageBytes + kWqCodeStage) + kWqBStages * kWqBStage +
+constexpr int kWqSmemBytes = kWqAStages * kAStageBytes + kWqCodeRing + kWqBStages * kWqBStage +
                              kWqEpiWarps * kStgWarpBytes + 512 /*SFP8 table*/ + 1024 /*align*/ + 512 /*barriers*/;
+static_assert(kWqSmemBytes <= 232448, "shared memory per CTA");
 
 struct WqProblem {
   int K;         // reduction length, multiple of 64
@@ -130,16 +144,20 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_constant__ WqParams P) {
   constexpr int kBlk = wq_block_bytes<FMT>();
+  constexpr int kCS = wq_code_stage<FMT>();
+  constexpr int kCStages = wq_cstages<FMT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sC = sA + kWqStages * kAStageBytes;
-  uint8_t* sB = sC + kWqStages * kWqCodeStage;
-  uint8_t* sStg = sB + kWqBStages * kWqBStage;
+  uint8_t* sB = sA + kWqAStages * kAStageBytes;
+  uint8_t* sC = sB + kWqBStages * kWqBStage;
+  uint8_t* sStg = sC + kWqCodeRing;
   uint16_t* s_lut = reinterpret_cast<uint16_t*>(sStg + kWqEpiWarps * kStgWarpBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_lut + 256);
-  uint64_t* empty = full + kWqStages;
-  uint64_t* bfull = empty + kWqStages;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(s_lut + 256);
+  uint64_t* aempty = afull + kWqAStages;
+  uint64_t* cfull = aempty + kWqAStages;
+  uint64_t* cempty = cfull + kWqMaxCStages;
+  uint64_t* bfull = cempty + kWqMaxCStages;
   uint64_t* bempty = bfull + kWqBStages;
   uint64_t* acc_full = bempty + kWqBStages;
   uint64_t* acc_empty = acc_full + 2;
@@ -153,12 +171,16 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr int kConv0 = 2 + kWqEpiWarps;          // first converter warp
-  constexpr int kCopy0 = kConv0 + kWqConvWarps;    // first copy warp
+  constexpr int kCopy0 = kConv0 + kWqConvWarps;    // first weight-block issuer warp
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kWqStages; ++s) {
-      mbar_init(&full[s], kWqNProd);          // one arrival (with its bytes) per issuing thread
-      mbar_init(&empty[s], 1 + kWqConvWarps);  // the MMAs have read A, the converters the codes
+    for (int s = 0; s < kWqAStages; ++s) {
+      mbar_init(&afull[s], 1);
+      mbar_init(&aempty[s], 1);  // the MMAs have read the A rows
+    }
+    for (int s = 0; s < kCStages; ++s) {
+      mbar_init(&cfull[s], kWqCopyWarps);   // one arrival (with its bytes) per block issuer
+      mbar_init(&cempty[s], kWqConvWarps);  // every converter warp has read the codes
     }
     for (int b = 0; b < kWqBStages; ++b) {
       mbar_init(&bfull[b], kWqConvWarps);
@@ -202,60 +224,22 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
              tile.n0 < 0 || tile.n0 >= pr.N || (tile.n0 & 127) || tile.kb0 != 0 || tile.kbn != 0 ||
              tile.rows1 != 0);
   };
-  // Copies of stage st (K block kb) of a tile, in a fixed order: the A rows,
-  // then the weight blocks (GATEUP: gate and up of the tile's 128 columns;
-  // DOWN: the one or two 128-row blocks of its up to 256 columns). Copy i
-  // belongs to issuing thread i % kWqNProd; returns grp's bytes and, with
-  // doit, issues them.
-  auto stage_copies = [&](int grp, bool doit, int st, int kb, const Tile& tile) -> uint32_t {
-    const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
-    const WqProblem& pr = P.prob[p];
-    const int wn = wq_tile_cols<GATEUP>(pr, tile.n0);
-    const bool a_small = P.a_small && tile.rows <= kASmallRows;
-    const int nb = (pr.N + 127) / 128, kbs = pr.K / kBK;
-    const int rb = tile.n0 >> 7;
-    uint32_t bytes = 0;
-    int i = 0;
-    auto mine = [&]() { return (i++ % kWqNProd) == grp; };
-    if (mine()) {
-      bytes += a_small ? kASmallBytes : kAStageBytes;
-      if (doit) tma_load_2d(sA + st * kAStageBytes, a_small ? &P.tmAs[p] : &P.tmA[p], &full[st], kb * kBK, tile.row0);
-    }
-    const int nblk = GATEUP ? 2 : (wn > 128 ? 2 : 1);
-    for (int q = 0; q < nblk; ++q) {
-      if (!mine()) continue;
-      bytes += kBlk;
-      if (!doit) continue;
-      const uint8_t* w = (GATEUP && q) ? pr.w1 : pr.w0;
-      const int row_blk = GATEUP ? rb : rb + q;
-      const size_t off = ((static_cast<size_t>(g) * nb + row_blk) * kbs + kb) * kBlk;
-      bulk_copy_g2s(sC + st * kWqCodeStage + q * 8192, w + off, kBlk, &full[st]);
-    }
-    return bytes;
-  };
-  auto arm_and_copy = [&](int grp, int st, int kb, const Tile& tile) {
-    const uint32_t b = stage_copies(grp, false, st, kb, tile);
-    if (b)
-      mbar_arrive_expect_tx(&full[st], b);
-    else
-      mbar_arrive(&full[st]);
-    stage_copies(grp, true, st, kb, tile);
-  };
-  auto drain_copies = [&](int s_now, uint32_t ph_now, int issued) {
+  // after an abort: let an issuer's copies in flight land before the CTA's memory goes away
+  auto drain_ring = [&](uint64_t* full_bars, int nst, int s_now, uint32_t ph_now, int issued) {
     int st = s_now;
     uint32_t sp = ph_now;
-    const int pending = issued < kWqStages ? issued : kWqStages;
+    const int pending = issued < nst ? issued : nst;
     for (int i = 0; i < pending; ++i) {
       if (--st < 0) {
-        st = kWqStages - 1;
+        st = nst - 1;
         sp ^= 1;
       }
       uint32_t dummy = 0;
-      mbar_wait(&full[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
+      mbar_wait(&full_bars[st], sp, reinterpret_cast<volatile int*>(&dummy), P.err, 100000000ull);
     }
   };
-  // A reader of the tile ring (MMA, epilogue, converter and copy warps): the
-  // next tile index, or -1 at the end / on abort.
+  // A reader of the tile ring (MMA, epilogue, converter and block-issuer
+  // warps): the next tile index, or -1 at the end / on abort.
   auto next_from_ring = [&](int& rs, uint32_t& rph, bool warp_wide) -> int {
     const bool got = mbar_wait(&tile_full[rs], rph, abort_flag, P.err);
     int ti = got ? tile_ring[rs] : -1;
@@ -269,7 +253,7 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
   };
 
   if (warp == 0) {
-    // -------------------------------------------------------- producer
+    // ------------------------------------------- producer (tiles, A rows)
     int s = 0, issued = 0;
     uint32_t ph = 0;
     int rs = 0;
@@ -302,20 +286,25 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
         }
         break;
       }
-      const int kb_end = P.prob[tile.pg >> 16].K / kBK;
+      const int p = tile.pg >> 16;
+      const bool a_small = P.a_small && tile.rows <= kASmallRows;
+      const int kb_end = P.prob[p].K / kBK;
       bool ok = true;
       for (int kb = 0; kb < kb_end; ++kb) {
         int waited = 1;
         if (lane == 0) {
-          waited = mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err);
-          if (waited) arm_and_copy(0, s, kb, tile);
+          waited = mbar_wait(&aempty[s], ph ^ 1, abort_flag, P.err);
+          if (waited) {
+            mbar_arrive_expect_tx(&afull[s], a_small ? kASmallBytes : kAStageBytes);
+            tma_load_2d(sA + s * kAStageBytes, a_small ? &P.tmAs[p] : &P.tmA[p], &afull[s], kb * kBK, tile.row0);
+          }
         }
         if (!__shfl_sync(0xffffffffu, waited, 0)) {
           ok = false;
           break;
         }
         ++issued;
-        if (++s == kWqStages) {
+        if (++s == kWqAStages) {
           s = 0;
           ph ^= 1;
         }
@@ -324,7 +313,7 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       ti = __shfl_sync(0xffffffffu, next, 0);
     }
     __syncwarp();
-    if (lane == 0 && *abort_flag) drain_copies(s, ph, issued);
+    if (lane == 0 && *abort_flag) drain_ring(afull, kWqAStages, s, ph, issued);
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
@@ -348,7 +337,7 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
         const uint32_t d_tmem = tmem_base + acc * kAccCols;
         bool ok = true;
         for (int kb = 0; kb < kb_end; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort_flag, P.err) || !mbar_wait(&bfull[b], bph, abort_flag, P.err)) {
+          if (!mbar_wait(&afull[s], ph, abort_flag, P.err) || !mbar_wait(&bfull[b], bph, abort_flag, P.err)) {
             ok = false;
             break;
           }
@@ -363,9 +352,9 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
             umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
           }
           any = true;
-          umma_commit(&empty[s]);   // A of this stage read
+          umma_commit(&aempty[s]);  // A of this stage read
           umma_commit(&bempty[b]);  // decoded weights read
-          if (++s == kWqStages) {
+          if (++s == kWqAStages) {
             s = 0;
             ph ^= 1;
           }
@@ -388,8 +377,10 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       }
     }
   } else if (warp >= kCopy0) {
-    // ------------------------------------------------------ copy warps
-    const int grp = warp - kCopy0 + 1;
+    // ------------------------------------------------- weight-block issuers
+    // Warp kCopy0 + q copies block q of every stage (GATEUP: q = 0 gate, 1 up;
+    // DOWN: the tile's first and, past 128 columns, second 128-row block).
+    const int q = warp - kCopy0;
     if (lane == 0) {
       int s = 0, issued = 0;
       uint32_t ph = 0;
@@ -400,23 +391,35 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
         if (ti < 0) break;
         const Tile tile = P.tiles[ti];
         if (!tile_ok(tile)) break;  // the producer reports it
-        const int kb_end = P.prob[tile.pg >> 16].K / kBK;
+        const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
+        const WqProblem& pr = P.prob[p];
+        const int wn = wq_tile_cols<GATEUP>(pr, tile.n0);
+        const bool mine = GATEUP || q == 0 || wn > 128;
+        const int nb = (pr.N + 127) / 128, kbs = pr.K / kBK;
+        const uint8_t* w = (GATEUP && q) ? pr.w1 : pr.w0;
+        const int row_blk = (tile.n0 >> 7) + (GATEUP ? 0 : q);
+        const uint8_t* src = w + (static_cast<size_t>(g) * nb + row_blk) * kbs * kBlk;
         bool ok = true;
-        for (int kb = 0; kb < kb_end; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, P.err)) {
+        for (int kb = 0; kb < kbs; ++kb) {
+          if (!mbar_wait(&cempty[s], ph ^ 1, abort_flag, P.err)) {
             ok = false;
             break;
           }
-          arm_and_copy(grp, s, kb, tile);
+          if (mine) {
+            mbar_arrive_expect_tx(&cfull[s], kBlk);
+            bulk_copy_g2s(sC + s * kCS + q * kBlk, src + static_cast<size_t>(kb) * kBlk, kBlk, &cfull[s]);
+          } else {
+            mbar_arrive(&cfull[s]);
+          }
           ++issued;
-          if (++s == kWqStages) {
+          if (++s == kCStages) {
             s = 0;
             ph ^= 1;
           }
         }
         if (!ok) break;
       }
-      if (*abort_flag) drain_copies(s, ph, issued);
+      if (*abort_flag) drain_ring(cfull, kCStages, s, ph, issued);
     }
   } else if (warp >= kConv0) {
     // ------------------------------------------------------- converters
@@ -439,51 +442,75 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       const int kb_end = pr.K / kBK;
       bool ok = true;
       for (int kb = 0; kb < kb_end; ++kb) {
-        const bool got = mbar_wait(&full[s], ph, abort_flag, P.err) && mbar_wait(&bempty[b], bph ^ 1, abort_flag, P.err);
+        const bool got =
+            mbar_wait(&cfull[s], ph, abort_flag, P.err) && mbar_wait(&bempty[b], bph ^ 1, abort_flag, P.err);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
-        const uint8_t* cs = sC + s * kWqCodeStage;
+        const uint8_t* cs = sC + s * kCS;
         uint8_t* bs = sB + b * kWqBStage;
-        for (int i = ct; i < rows_b * 8; i += kWqConvThreads) {
+        // A thread's (up to) kIt items of the stage: all code loads first, then
+        // the decodes, then the stores, so that the shared-memory latencies of
+        // the items overlap instead of adding up.
+        constexpr int kIt = 256 * 8 / kWqConvThreads;
+        const int n_items = rows_b * 8;
+        uint32_t w0[kIt], w1[kIt];
+        float dsc[kIt];
+#pragma unroll
+        for (int j = 0; j < kIt; ++j) {
+          const int i = ct + j * kWqConvThreads;
+          if (i >= n_items) continue;
           const int r = i >> 3, c = i & 7;
           // which copied block, and which of its rows, holds B row r
           const int blk = GATEUP ? (r >= wn) : (r >> 7);
           const int sr = GATEUP ? (r >= wn ? r - wn : r) : (r & 127);
-          const uint8_t* src = cs + blk * 8192;
-          uint4 o;
+          const uint8_t* src = cs + blk * kBlk;
           if (FMT == kWfSfp8) {
             const uint2 raw = *reinterpret_cast<const uint2*>(src + sr * 64 + 8 * c);
-            const uint32_t w[2] = {raw.x, raw.y};
-            uint32_t v[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t word = w[j >> 1] >> (16 * (j & 1));
-              v[j] = static_cast<uint32_t>(s_lut[word & 0xFFu]) | (static_cast<uint32_t>(s_lut[(word >> 8) & 0xFFu]) << 16);
-            }
-            o = make_uint4(v[0], v[1], v[2], v[3]);
+            w0[j] = raw.x;
+            w1[j] = raw.y;
           } else {
-            const uint32_t q = *reinterpret_cast<const uint32_t*>(src + sr * 32 + 4 * c);
-            const float d = __half2float(*reinterpret_cast<const __half*>(src + 4096 + sr * 4 + 2 * (c >> 2)));
-            uint32_t v[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float lo = __int2float_rn(static_cast<int>((q >> (8 * j)) & 15u) - 8);
-              const float hi = __int2float_rn(static_cast<int>((q >> (8 * j + 4)) & 15u) - 8);
-              v[j] = pack_bf16x2(__fmul_rn(lo, d), __fmul_rn(hi, d));
-            }
-            o = make_uint4(v[0], v[1], v[2], v[3]);
+            w0[j] = *reinterpret_cast<const uint32_t*>(src + sr * 32 + 4 * c);
+            dsc[j] = __half2float(*reinterpret_cast<const __half*>(src + 4096 + sr * 4 + 2 * (c >> 2)));
           }
-          *reinterpret_cast<uint4*>(bs + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = o;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cempty[s]);  // this warp is done with the stage's codes
+        uint4 o[kIt];
+#pragma unroll
+        for (int j = 0; j < kIt; ++j) {
+          const int i = ct + j * kWqConvThreads;
+          if (i >= n_items) continue;
+          uint32_t v[4];
+          if (FMT == kWfSfp8) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const uint32_t word = (qq < 2 ? w0[j] : w1[j]) >> (16 * (qq & 1));
+              v[qq] = static_cast<uint32_t>(s_lut[word & 0xFFu]) |
+                      (static_cast<uint32_t>(s_lut[(word >> 8) & 0xFFu]) << 16);
+            }
+          } else {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const float lo = __int2float_rn(static_cast<int>((w0[j] >> (8 * qq)) & 15u) - 8);
+              const float hi = __int2float_rn(static_cast<int>((w0[j] >> (8 * qq + 4)) & 15u) - 8);
+              v[qq] = pack_bf16x2(__fmul_rn(lo, dsc[j]), __fmul_rn(hi, dsc[j]));
+            }
+          }
+          o[j] = make_uint4(v[0], v[1], v[2], v[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < kIt; ++j) {
+          const int i = ct + j * kWqConvThreads;
+          if (i >= n_items) continue;
+          const int r = i >> 3, c = i & 7;
+          *reinterpret_cast<uint4*>(bs + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = o[j];
         }
         fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bfull[b]);
-          mbar_arrive(&empty[s]);  // this warp is done with the stage's codes
-        }
-        if (++s == kWqStages) {
+        if (lane == 0) mbar_arrive(&bfull[b]);
+        if (++s == kCStages) {
           s = 0;
           ph ^= 1;
         }

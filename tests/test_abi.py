@@ -40,8 +40,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert B.moe_status_string(code).startswith("MOE_")
+    assert B.moe_status_string(B.MOE_ERR_GUARD) == "MOE_ERR_GUARD"
 
 
 def test_workspace_sizes(lib):
@@ -126,3 +127,15 @@ def test_round_bf16_validation(lib):
     assert f(16, 1 << 20, 12, None) == B.MOE_ERR_INVALID_ARG  # n not a multiple of 8
     assert f(20, 1 << 20, 8, None) == B.MOE_ERR_ALIGNMENT
     assert f(1 << 20, (1 << 20) + 16, 8, None) == B.MOE_ERR_INVALID_ARG  # overlap
+
+
+def test_workspace_guard_layout(lib):
+    """The layout ends in 256 guard bytes after every data region."""
+    for T in (1, 64, 4096):
+        lay = B.moe_workspace_layout(B.make_params(T))
+        assert lay.guard % 256 == 0 and lay.total_bytes == lay.guard + 256
+        assert lay.guard >= max(lay.x_perm, lay.h, lay.y, lay.hs, lay.s, lay.x_norm, lay.token_of)
+    p = B.make_params(8)
+    assert lib.moe_workspace_guard_check(ctypes.byref(p), None) == B.MOE_ERR_INVALID_ARG  # no workspace
+    p = B.make_params(8, workspace=1 << 20, workspace_bytes=64)
+    assert lib.moe_workspace_guard_check(ctypes.byref(p), None) == B.MOE_ERR_WORKSPACE
