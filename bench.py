@@ -591,16 +591,21 @@ def run_stack(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        B.moe_profile_begin([dominant])
         e0.record(stream)
         for _ in range(args.steps):
             stk.stack_forward(st, x, bufs, ws, stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        per_kernel = B.moe_profile_end()
     barrier(world)
     ms = reduce_max(e0.elapsed_time(e1), world)
     agg = aggregate(T, args.steps, ms, world)
+    # the dominant kernel's own duration, in a pass of its own: an event
+    # between two kernels ends their programmatic-launch overlap
+    B.moe_profile_begin([dominant])
+    for _ in range(args.steps):
+        stk.stack_forward(st, x, bufs, ws, stream)
+    torch.cuda.synchronize()
+    per_kernel = B.moe_profile_end()
     if B.moe_get_device_status() != B.MOE_OK:
         raise RuntimeError("device status after the timed region")
 
@@ -920,16 +925,19 @@ def run_dense(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        B.moe_profile_begin([dominant])
         e0.record(stream)
         for _ in range(args.steps):
             B.check(B.moe_dense_ffn_forward(p, stream), "dense")
         e1.record(stream)
         torch.cuda.synchronize()
-        per_kernel = B.moe_profile_end()
     barrier(world)
     ms = reduce_max(e0.elapsed_time(e1), world)
     agg = aggregate(T, args.steps, ms, world)
+    B.moe_profile_begin([dominant])  # the dominant kernel alone, outside the timed region
+    for _ in range(args.steps):
+        B.check(B.moe_dense_ffn_forward(p, stream), "dense")
+    torch.cuda.synchronize()
+    per_kernel = B.moe_profile_end()
     if B.moe_get_device_status() != B.MOE_OK:
         raise RuntimeError("device status after the timed region")
     # end to end through the public call: pinned host x in, host out back

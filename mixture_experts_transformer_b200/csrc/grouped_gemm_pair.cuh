@@ -27,6 +27,15 @@
 
 namespace moe {
 
+// Arrive without release semantics, for the barrier that hands the peer's
+// MMA thread back an accumulator: its tcgen05.ld results are in registers
+// (tcgen05.wait::ld and tcgen05.fence::before_thread_sync come first), and a
+// release at cluster scope would first wait for every global store of the
+// epilogue to complete.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 constexpr int kP2Stages = 6;
 constexpr int kP2AStage = kBM * kBK * 2;        // 16 KB: this CTA's 128 rows
 constexpr int kP2BStage = 2 * kBChunkBytes;     // 16 KB: this CTA's half of B (<= 128 columns)
@@ -270,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_even + 8u * acc);
+      if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_even + 8u * acc);
       if (++acc == 2) {
         acc = 0;
         acc_ph ^= 1;

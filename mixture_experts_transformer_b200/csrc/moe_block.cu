@@ -509,7 +509,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256,
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256, 128,
                                      (allow_pairs && paired_gateup(d)) ? 1 : 0,
                                      (pairs || (allow_pairs && paired_down(d))) ? 1 : 0, d.e0, d.el);
     MOE_TRY(ls_.done(le_));
@@ -785,7 +785,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
     const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
-                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 0, 0, 0, d.E);
+                                     reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 128, 0, 0, 0, d.E);
     MOE_TRY(ls_.done(le_));
   }
   {
@@ -813,6 +813,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   gu.nprob = 2;
   gu.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_gu);
   gu.num_tiles = &counts->gateup;
+  gu.next_tile = &counts->next_gateup;
   gu.err = s->err;
   {
     LaunchScope ls_(kKFp4GateUp, st);
@@ -837,6 +838,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   dn.nprob = 2;
   dn.tiles = reinterpret_cast<const Tile*>(ws + L.tiles_dn);
   dn.num_tiles = &counts->down;
+  dn.next_tile = &counts->next_down;
   dn.err = s->err;
   {
     LaunchScope ls_(kKFp4Down, st);

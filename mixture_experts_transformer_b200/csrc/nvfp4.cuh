@@ -255,7 +255,7 @@ __host__ __device__ constexpr int f4_threads() {
   return kF4Threads + 128;
 }
 constexpr int kF4StgWarpBytes = 1024;            // epilogue staging per warp (32 rows x 32 B)
-constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 8 * kF4StgWarpBytes + 1024 + 256;
+constexpr int kF4SmemBytes = kF4Stages * (kF4ABytes + kF4BBytes + 3 * kF4SfBytes) + 8 * kF4StgWarpBytes + 1024 + 512;
 
 struct Fp4Problem {
   int K;          // multiple of 64
@@ -284,6 +284,7 @@ struct Fp4Params {
   int nprob;
   const Tile* tiles;
   const int32_t* num_tiles;
+  int32_t* next_tile;   // work counter (zero at launch): tiles go to CTAs as they free up
   uint32_t* err;
 };
 
@@ -355,8 +356,11 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint64_t* sf_ready = drain + 1;  // a stage's scale atoms are in TMEM (one arrival per scale warp)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_ready + kF4Stages);
+  uint64_t* tile_full = sf_ready + kF4Stages;
+  uint64_t* tile_empty = tile_full + kTileRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_empty + kTileRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* tile_ring = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -371,6 +375,10 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
       mbar_init(&acc_empty[a], 8);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < kTileRing; ++r) {
+      mbar_init(&tile_full[r], 1);
+      mbar_init(&tile_empty[r], 1 + 8 + 4);  // MMA thread, epilogue and scale warps read each index
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -391,13 +399,44 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait_then_release();
   const int num_tiles = *P.num_tiles;
+  // The producer takes tile indices from the work counter and publishes them
+  // in the ring (-1 ends the work); the other roles read them in order. A
+  // consumer's next index: lane 0 of its warp waits, the warp shares it
+  // (-1 as well when the wait gave up).
+  int rs = 0;
+  uint32_t rph = 0;
+  auto next_tile = [&](bool whole_warp) -> int {
+    int ti = -1;
+    if (lane == 0) {
+      if (mbar_wait(&tile_full[rs], rph, abort_flag, P.err)) {
+        ti = tile_ring[rs];
+        mbar_arrive(&tile_empty[rs]);
+      }
+    }
+    if (whole_warp) ti = __shfl_sync(0xffffffffu, ti, 0);
+    if (++rs == kTileRing) {
+      rs = 0;
+      rph ^= 1;
+    }
+    return ti;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ TMA producer
       int s = 0, issued = 0;
       uint32_t ph = 0;
-      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      int ti = atomicAdd(P.next_tile, 1);
+      while (true) {
+        if (!mbar_wait(&tile_empty[rs], rph ^ 1, abort_flag, P.err)) break;
+        tile_ring[rs] = ti < num_tiles ? ti : -1;
+        mbar_arrive(&tile_full[rs]);
+        if (++rs == kTileRing) {
+          rs = 0;
+          rph ^= 1;
+        }
+        if (ti >= num_tiles) break;
+        const int next = atomicAdd(P.next_tile, 1);  // its latency hides behind this tile's loads
         const Tile tile = P.tiles[ti];
         const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
         if (p >= P.nprob) {
@@ -449,6 +488,7 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
           }
         }
         if (!ok) break;
+        ti = next;
       }
       if (*abort_flag) {
         int st = s;
@@ -472,7 +512,9 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
       bool any = false;
       const uint32_t idesc = idesc_nvf4_m128(128);
       const uint32_t idesc256 = idesc_nvf4_m128(256);
-      for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+      while (true) {
+        const int ti = next_tile(false);
+        if (ti < 0) break;
         const Tile tile = P.tiles[ti];
         const int p = tile.pg >> 16;
         if (p >= P.nprob) break;
@@ -544,7 +586,9 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int s = 0, slot = 0;
     uint32_t ph = 0;
-    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+    while (true) {
+      const int ti = next_tile(true);
+      if (ti < 0) break;
       const Tile tile = P.tiles[ti];
       const int p = tile.pg >> 16;
       if (p >= P.nprob) break;
@@ -589,7 +633,9 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
     const int r = quarter * 32 + lane;
     int acc_i = 0;
     uint32_t acc_ph = 0;
-    for (int ti = blockIdx.x; ti < num_tiles; ti += gridDim.x) {
+    while (true) {
+      const int ti = next_tile(true);
+      if (ti < 0) break;
       const Tile tile = P.tiles[ti];
       const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
       if (p >= P.nprob) break;

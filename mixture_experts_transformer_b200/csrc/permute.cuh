@@ -50,7 +50,7 @@ __global__ void build_masks_kernel(const int32_t* __restrict__ idx, int T, int k
 
 // One CTA of 1024 threads: thread (e, seg) walks one eighth of the 32-token
 // chunks of expert e. Produces cnt, off, base[c][e] and the tile lists
-// (gate|up tiles 128 output columns per projection, down tiles dn_cols wide):
+// (gate|up tiles gu_cols output columns per projection, down tiles dn_cols wide):
 // shared-MLP tiles first (problem 1), then expert tiles (problem 0) expert by
 // expert, column tile, then row tile, so CTAs that run at the same time read
 // the same weight columns and share them through L2.
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
                                                                   Tile* __restrict__ tiles_gu,
                                                                   Tile* __restrict__ tiles_dn,
                                                                   TileCounts* __restrict__ counts, int padded,
-                                                                  int dn_cols, int pair_gu, int pair_dn,
+                                                                  int dn_cols, int gu_cols, int pair_gu, int pair_dn,
                                                                   int e_begin, int e_count) {
   __shared__ int s_seg[kScanSegs][128];
   __shared__ int s_off[129];
@@ -149,10 +149,10 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   if (threadIdx.x == 0) off_out[E] = s_off[E];
 
   // A tile takes one 128-row block, or (paired GEMM) two consecutive blocks of
-  // the same expert and column tile. Gate|up tiles are 128 output columns per
-  // projection, down tiles dn_cols wide.
+  // the same expert and column tile. Gate|up tiles are gu_cols output columns
+  // per projection, down tiles dn_cols wide.
   const int mt_sh = (T + kBM - 1) / kBM;
-  const int nt_gu = (F + 127) / 128;
+  const int nt_gu = (F + gu_cols - 1) / gu_cols;
   const int nt_dn = (D + dn_cols - 1) / dn_cols;
   auto emit = [&](Tile* tiles, int pair, int ncol_sh, int ncol, int cw) -> int {
     const int mstep = pair ? 2 : 1;
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     }
     return n_sh + n_e;
   };
-  const int n_gu = emit(tiles_gu, pair_gu, (S + 127) / 128, nt_gu, 128);
+  const int n_gu = emit(tiles_gu, pair_gu, (S + gu_cols - 1) / gu_cols, nt_gu, gu_cols);
   const int n_dn = emit(tiles_dn, pair_dn, (D + dn_cols - 1) / dn_cols, nt_dn, dn_cols);
   if (threadIdx.x == 0) {
     counts->gateup = n_gu;

@@ -80,7 +80,7 @@ __host__ __device__ constexpr int wq_cstages() {
 }
 constexpr int kWqBStage = 256 * kBK * 2;        // 256 weight rows x 64 K bf16
 constexpr int kWqSmemBytes = kWqAStages * kAStageBytes + kWqCodeRing + kWqBStages * kWqBStage +
-                             kWqEpiWarps * kStgWarpBytes + 512 /*SFP8 table*/ + 1024 /*align*/ + 512 /*barriers*/;
+                             kWqEpiWarps * kStgWarpBytes + 1024 /*align*/ + 512 /*barriers*/;
 static_assert(kWqSmemBytes <= 232448, "shared memory per CTA");
 
 struct WqProblem {
@@ -128,6 +128,30 @@ __host__ __device__ inline uint16_t sfp8_bf16_bits(uint32_t code) {
   return static_cast<uint16_t>(bits | ((code & 0x80u) << 8));
 }
 
+// Bytes 0 and 2 of x, each replaced by copies of its top bit, in both bytes
+// of their 16-bit halves: prmt's sign-replicating selectors (CUDA's
+// __byte_perm keeps only the byte-select bits of a selector).
+__device__ __forceinline__ uint32_t replicate_top_bits_b02(uint32_t x) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, 0xAA88;" : "=r"(r) : "r"(x));
+  return r;
+}
+
+// Two SFP8 codes, in bytes 0 and 2 of v (bytes 1 and 3 are ignored), to two
+// bf16 bit patterns: m >= 64 -> 0x3800 + 16 m, 1 <= m < 64 -> 0x3400 + 32 m,
+// m = 0 -> 0, sign to bit 15. Both candidates are computed in packed 16-bit
+// lanes and selected by per-lane masks spread from one bit of each code
+// (bit 6: m >= 64; the carry of m + 127 into bit 7: m != 0). Equal to
+// sfp8_bf16_bits for all 2^16 code pairs.
+__device__ __forceinline__ uint32_t sfp8x2_to_bf16x2(uint32_t v) {
+  const uint32_t m = v & 0x007F007Fu;
+  const uint32_t lg = m * 16u + 0x38003800u;
+  const uint32_t sm = m * 32u + 0x34003400u;
+  const uint32_t big = replicate_top_bits_b02(v << 1);
+  const uint32_t nz = replicate_top_bits_b02(m + 0x007F007Fu);
+  return (((lg & big) | (sm & ~big)) & nz) | ((v << 8) & 0x80008000u);
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -152,8 +176,7 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
   uint8_t* sB = sA + kWqAStages * kAStageBytes;
   uint8_t* sC = sB + kWqBStages * kWqBStage;
   uint8_t* sStg = sC + kWqCodeRing;
-  uint16_t* s_lut = reinterpret_cast<uint16_t*>(sStg + kWqEpiWarps * kStgWarpBytes);
-  uint64_t* afull = reinterpret_cast<uint64_t*>(s_lut + 256);
+  uint64_t* afull = reinterpret_cast<uint64_t*>(sStg + kWqEpiWarps * kStgWarpBytes);
   uint64_t* aempty = afull + kWqAStages;
   uint64_t* cfull = aempty + kWqAStages;
   uint64_t* cempty = cfull + kWqMaxCStages;
@@ -198,7 +221,6 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (FMT == kWfSfp8 && threadIdx.x < 256) s_lut[threadIdx.x] = sfp8_bf16_bits(threadIdx.x);
   if (warp == 0 && lane == 0) {
     for (int p = 0; p < P.nprob; ++p) {
       tma_prefetch_desc(&P.tmA[p]);
@@ -484,18 +506,27 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
           if (i >= n_items) continue;
           uint32_t v[4];
           if (FMT == kWfSfp8) {
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const uint32_t word = (qq < 2 ? w0[j] : w1[j]) >> (16 * (qq & 1));
-              v[qq] = static_cast<uint32_t>(s_lut[word & 0xFFu]) |
-                      (static_cast<uint32_t>(s_lut[(word >> 8) & 0xFFu]) << 16);
-            }
+            // two codes per 32-bit word (one per 16-bit half), decoded together
+            v[0] = sfp8x2_to_bf16x2(__byte_perm(w0[j], 0u, 0x4140));
+            v[1] = sfp8x2_to_bf16x2(__byte_perm(w0[j], 0u, 0x4342));
+            v[2] = sfp8x2_to_bf16x2(__byte_perm(w1[j], 0u, 0x4140));
+            v[3] = sfp8x2_to_bf16x2(__byte_perm(w1[j], 0u, 0x4342));
           } else {
+            // A nibble q at bit 8 (12) of a word, or'ed into the mantissa of
+            // 1.0, is the float f = 1 + q 2^-15 (1 + q 2^-11); one fma
+            // f A + B with A = d 2^15, B = -d (2^15 + 8) (2^11 for bit 12)
+            // gives (q - 8) d: A and B are exact (at most 13 x 11 significant
+            // bits), and so is (q - 8) d (4 x 11), so the fma's one rounding
+            // leaves it exact; then one rounding to bf16.
+            const float d = dsc[j];
+            const float a8 = __fmul_rn(d, 32768.0f), b8 = __fmul_rn(d, -32776.0f);
+            const float a12 = __fmul_rn(d, 2048.0f), b12 = __fmul_rn(d, -2056.0f);
+            const uint32_t x[4] = {w0[j] << 8, w0[j], w0[j] >> 8, w0[j] >> 16};  // elements 2qq, 2qq + 1 at bits 8, 12
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
-              const float lo = __int2float_rn(static_cast<int>((w0[j] >> (8 * qq)) & 15u) - 8);
-              const float hi = __int2float_rn(static_cast<int>((w0[j] >> (8 * qq + 4)) & 15u) - 8);
-              v[qq] = pack_bf16x2(__fmul_rn(lo, dsc[j]), __fmul_rn(hi, dsc[j]));
+              const float lo = __uint_as_float((x[qq] & 0x00000F00u) | 0x3F800000u);
+              const float hi = __uint_as_float((x[qq] & 0x0000F000u) | 0x3F800000u);
+              v[qq] = pack_bf16x2(__fmaf_rn(lo, a8, b8), __fmaf_rn(hi, a12, b12));
             }
           }
           o[j] = make_uint4(v[0], v[1], v[2], v[3]);
