@@ -436,8 +436,10 @@ moe_status moe_nvfp4_calibrate(const moe_params* p, float* amax, float* scales, 
  * transposed weight in 128-row blocks and 64-deep K blocks:
  *   SFP8: q [G][ceil(N/128)][K/64][128 rows x 64 code bytes]; scale [G] fp32
  *   Q4_0: q [G][ceil(N/128)][K/64][128 rows x 32 bytes | 128 rows x 2 fp16 d]
- *         (element 2j of a row's 64 in the low nibble of byte j; the row's two
- *         scales cover K 0-31 and 32-63); scale unused (NULL)
+ *         (element 2i of a 16-byte piece in the low nibble of its byte i; the
+ *         row's two scales cover K 0-31 and 32-63); scale unused (NULL)
+ * A row's codes are 16-byte pieces in K order, piece j of row r stored at
+ * position j ^ ((r >> 1) & 3) (SFP8) or j ^ ((r >> 2) & 1) (Q4_0) of the row.
  * Rows past N hold zeros.
  */
 #define MOE_WFMT_SFP8 1

@@ -1,12 +1,15 @@
 // Grouped GEMM with the weights in a weight-only format, SFP8 or Q4_0 (the
 // formats the pages name by their footprint; readings below), activations in
 // bf16. The tensor cores take bf16 operands, so converter warps decode each
-// stage's weight codes into bf16 in shared memory, in the 128-byte-swizzled
-// K-major layout the MMA reads; everything else is the grouped GEMM of
-// grouped_gemm.cuh (same tile lists, epilogues and barriers).
+// stage's weight codes into bf16 and write them straight into tensor memory,
+// where the MMA reads them as its A operand: the product is computed
+// transposed, D^T = W^T X^T, with the tile's 128 weight columns as M (TMEM
+// lanes) and its token rows as N (rounded up to 16). The decoded weights never
+// pass through shared memory, which at small batches would otherwise carry
+// three times the code bytes (codes in, bf16 out, bf16 read by the MMA).
 //
-//   GATEUP: h[row, n] = gelu_tanh(A Wg^)[row, n] * (A Wu^)[row, n]   (bf16 out)
-//   DOWN:   y[row, n] = (A Wd^)[row, n]                              (bf16 or fp32 out)
+//   GATEUP: h[row, n] = gelu_tanh(X Wg^)[row, n] * (X Wu^)[row, n]   (bf16 out)
+//   DOWN:   y[row, n] = (X Wd^)[row, n]                              (bf16 or fp32 out)
 //
 // Formats (one [K, N] Linear; weights quantised along K, their input axis):
 //   SFP8 - sign bit and a 7-bit magnitude code m: 0 is zero; m in [1, 63] is
@@ -24,27 +27,29 @@
 // that a stage brings it with one bulk copy:
 //   SFP8: [G][ceil(N/128)][K/64][128 rows x 64 B codes]                     8192 B
 //   Q4_0: [G][ceil(N/128)][K/64][128 rows x 32 B codes | 128 rows x 2 fp16]  4608 B
-// (Q4_0: element 2j of a row's 64 in the low nibble of byte j; a row's two
+// A row's codes are 16-byte pieces in K order, piece j stored at position
+// j ^ ((r >> 1) & 3) (SFP8) or j ^ ((r >> 2) & 1) (Q4_0) of row r, so that the
+// 32 rows a converter warp reads at once spread over all shared-memory banks.
+// (Q4_0: element 2i of a piece in the low nibble of its byte i; a row's two
 // scales cover K 0-31 and 32-63 of the block.) Rows past N hold zeros.
 //
 // Roles (512 threads, one CTA per SM; 16 warps, so 4 per SM sub-partition):
 //   warp 0        producer: tiles from the work counter into the tile ring,
-//                 and the A rows of every stage into the A ring
-//   warp 1        MMA issuer: waits for a stage's A rows and decoded weights,
-//                 4 x tcgen05.mma (K = 16), frees both
-//   warps 2..5    epilogue, one per TMEM lane quarter
-//   warps 6..13   converters: a stage's codes -> bf16 weights (K-major, 128-byte
-//                 swizzle) in a 2-deep ring, then a proxy fence and arrival
+//                 and the token rows of every stage into the X ring (TMA)
+//   warp 1        MMA issuer: waits for a stage's token rows and decoded
+//                 weights, 4 x (one or two) tcgen05.mma (K = 16, A in TMEM)
+//   warps 2..5    epilogue, one per TMEM lane quarter (32 weight columns)
+//   warps 6..13   converters: warp 6 + 4 b + q decodes rows 32 q .. 32 q + 31
+//                 of weight block b of a stage (one row per thread) into TMEM
+//                 lanes 32 q .. (tcgen05.st), then arrives
 //   warps 14, 15  the weight blocks of every stage (block 0 and block 1) into
-//                 the code ring (one thread issues ~2.2 M copies per second,
-//                 so the A copy and the two block copies go to three threads)
-// The rings are separate: A slots are freed by the MMAs, code slots by the
-// converters as soon as they have read them. The weight stream, which carries
-// nearly all of the bytes at small batches, so runs as far ahead as the code
-// ring is deep (5 stages of SFP8, 8 of Q4_0), not only as far as the
-// converters may run ahead of the MMAs.
-// Shared memory: A ring 4 x 16 KB, code ring 80 KB, decoded weights 2 x 32 KB.
-// TMEM: 2 accumulators x 256 columns.
+//                 the code ring by bulk copy
+// Each ring is freed by its reader: X slots and TMEM weight stages by the MMAs'
+// commits, code slots by the converters once they have read them, so the
+// weight stream runs as far ahead as the code ring is deep.
+// Shared memory: X ring 4 x 16 KB, code ring 128 KB. TMEM: the two
+// accumulators D0, D1 (128 columns each: block 0 and block 1 of the tile)
+// and 4 stages of decoded weights (32 columns per block).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -61,15 +66,18 @@ __host__ __device__ constexpr int wq_block_bytes() {
   return FMT == kWfSfp8 ? 8192 : 4608;
 }
 
-constexpr int kWqAStages = 4;
-constexpr int kWqBStages = 2;
+constexpr int kWqXStages = 4;     // token-row stages (shared memory)
+constexpr int kWqTStages = 4;     // decoded-weight stages (TMEM)
 constexpr int kWqEpiWarps = 4;
 constexpr int kWqConvWarps = 8;
 constexpr int kWqCopyWarps = 2;  // the two weight-block issuers
 constexpr int kWqThreads = 32 * (2 + kWqEpiWarps + kWqConvWarps + kWqCopyWarps);
-constexpr int kWqConvThreads = 32 * kWqConvWarps;
-constexpr int kWqCodeRing = 80 * 1024;          // code ring bytes
-constexpr int kWqMaxCStages = 8;
+constexpr int kWqCodeRing = 128 * 1024;         // code ring bytes
+constexpr int kWqMaxCStages = 16;
+constexpr uint32_t kWqDCols = 128;               // one accumulator: 128 lanes x up to 128 token columns
+constexpr uint32_t kWqTCol0 = 2 * kWqDCols;      // first TMEM column of the weight stages
+constexpr uint32_t kWqTStageCols = 64;           // a stage: block 0 at +0, block 1 at +32 (64 bf16 of K each)
+static_assert(kWqTCol0 + kWqTStages * kWqTStageCols <= 512, "TMEM columns");
 template <int FMT>
 __host__ __device__ constexpr int wq_code_stage() {  // two 128-row weight blocks
   return 2 * wq_block_bytes<FMT>();
@@ -78,9 +86,8 @@ template <int FMT>
 __host__ __device__ constexpr int wq_cstages() {
   return kWqCodeRing / wq_code_stage<FMT>() < kWqMaxCStages ? kWqCodeRing / wq_code_stage<FMT>() : kWqMaxCStages;
 }
-constexpr int kWqBStage = 256 * kBK * 2;        // 256 weight rows x 64 K bf16
-constexpr int kWqSmemBytes = kWqAStages * kAStageBytes + kWqCodeRing + kWqBStages * kWqBStage +
-                             kWqEpiWarps * kStgWarpBytes + 1024 /*align*/ + 512 /*barriers*/;
+constexpr int kWqSmemBytes = kWqXStages * kAStageBytes + kWqCodeRing + kWqEpiWarps * kStgWarpBytes +
+                             1024 /*align*/ + 1024 /*barriers*/;
 static_assert(kWqSmemBytes <= 232448, "shared memory per CTA");
 
 struct WqProblem {
@@ -165,6 +172,119 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
                : "memory");
 }
 
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait_all() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// tcgen05.mma kind::f16 with A in tensor memory (M = 128 lanes, 16 bf16 of K
+// packed in 8 columns) and B from a shared-memory descriptor.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Epilogue stores of a transposed accumulator: thread `lane` holds column
+// `lane` of 32 output rows (a[i] = row i). The values go through the warp's
+// 4 KB staging buffer as fp32 [32 rows][32 columns] (16-byte pieces XOR-
+// swizzled by row, conflict-free both ways), then the warp stores 16 bytes
+// per lane along the rows. Rows at or past rows_valid are not stored.
+__device__ __forceinline__ void stage_cols_f32x32(uint8_t* stg, const uint32_t (&a)[32], int lane) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    *reinterpret_cast<uint32_t*>(stg + i * 128 + (((lane >> 2) ^ (i & 7)) << 4) + (lane & 3) * 4) = a[i];
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_cols_f32x32(uint8_t* stg, const uint32_t (&a)[32], int lane, float* base,
+                                                  size_t ldo, int rows_valid) {
+  stage_cols_f32x32(stg, a, lane);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int row = it * 4 + (lane >> 3), c = lane & 7;  // 8 pieces of 16 B per row
+    const uint4 v = *reinterpret_cast<const uint4*>(stg + row * 128 + ((c ^ (row & 7)) << 4));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + c * 4) = v;
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void store_cols_bf16x32(uint8_t* stg, const uint32_t (&a)[32], int lane,
+                                                   __nv_bfloat16* base, size_t ldo, int rows_valid) {
+  stage_cols_f32x32(stg, a, lane);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int row = it * 8 + (lane >> 2), v = lane & 3;  // 4 pieces of 8 bf16 per row
+    const uint4 lo = *reinterpret_cast<const uint4*>(stg + row * 128 + (((2 * v) ^ (row & 7)) << 4));
+    const uint4 hi = *reinterpret_cast<const uint4*>(stg + row * 128 + (((2 * v + 1) ^ (row & 7)) << 4));
+    const uint4 pk = make_uint4(pack_bf16x2(__uint_as_float(lo.x), __uint_as_float(lo.y)),
+                                pack_bf16x2(__uint_as_float(lo.z), __uint_as_float(lo.w)),
+                                pack_bf16x2(__uint_as_float(hi.x), __uint_as_float(hi.y)),
+                                pack_bf16x2(__uint_as_float(hi.z), __uint_as_float(hi.w)));
+    if (row < rows_valid) *reinterpret_cast<uint4*>(base + static_cast<size_t>(row) * ldo + v * 8) = pk;
+  }
+  __syncwarp();
+}
+
+// Decoded row of one weight block for one stage: the 64 K of row r (codes at
+// `blk`, swizzled as stored) as 32 packed bf16x2 words, word c = K 2c, 2c + 1.
+template <int FMT>
+__device__ __forceinline__ void wq_decode_row(const uint8_t* blk, int r, uint32_t (&out)[32]) {
+  if (FMT == kWfSfp8) {
+    const uint8_t* row = blk + r * 64;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ ((r >> 1) & 3)) << 4));  // K 16 j .. 16 j + 15
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        out[8 * j + 2 * i] = sfp8x2_to_bf16x2(__byte_perm(ws[i], 0u, 0x4140));
+        out[8 * j + 2 * i + 1] = sfp8x2_to_bf16x2(__byte_perm(ws[i], 0u, 0x4342));
+      }
+    }
+  } else {
+    const uint8_t* row = blk + r * 32;
+    const __half2 dd = *reinterpret_cast<const __half2*>(blk + 4096 + r * 4);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      // A nibble q at bit 8 (12) of a word, or'ed into the mantissa of 1.0, is
+      // the float f = 1 + q 2^-15 (1 + q 2^-11); one fma f A + B with
+      // A = d 2^15, B = -d (2^15 + 8) (2^11 for bit 12) gives (q - 8) d: A and
+      // B are exact (at most 13 x 11 significant bits), and so is (q - 8) d
+      // (4 x 11), so the fma's one rounding leaves it exact; then one
+      // rounding to bf16.
+      const float d = __half2float(j ? dd.y : dd.x);
+      const float a8 = __fmul_rn(d, 32768.0f), b8 = __fmul_rn(d, -32776.0f);
+      const float a12 = __fmul_rn(d, 2048.0f), b12 = __fmul_rn(d, -2056.0f);
+      const uint4 w = *reinterpret_cast<const uint4*>(row + ((j ^ ((r >> 2) & 1)) << 4));  // K 32 j .. 32 j + 31
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t x[4] = {ws[i] << 8, ws[i], ws[i] >> 8, ws[i] >> 16};  // elements 2qq, 2qq + 1 at bits 8, 12
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const float lo = __uint_as_float((x[qq] & 0x00000F00u) | 0x3F800000u);
+          const float hi = __uint_as_float((x[qq] & 0x0000F000u) | 0x3F800000u);
+          out[16 * j + 4 * i + qq] = pack_bf16x2(__fmaf_rn(lo, a8, b8), __fmaf_rn(hi, a12, b12));
+        }
+      }
+    }
+  }
+}
+
 template <int FMT, bool GATEUP>
 __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_constant__ WqParams P) {
   constexpr int kBlk = wq_block_bytes<FMT>();
@@ -172,19 +292,18 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
   constexpr int kCStages = wq_cstages<FMT>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + kWqAStages * kAStageBytes;
-  uint8_t* sC = sB + kWqBStages * kWqBStage;
+  uint8_t* sX = smem;
+  uint8_t* sC = sX + kWqXStages * kAStageBytes;
   uint8_t* sStg = sC + kWqCodeRing;
-  uint64_t* afull = reinterpret_cast<uint64_t*>(sStg + kWqEpiWarps * kStgWarpBytes);
-  uint64_t* aempty = afull + kWqAStages;
-  uint64_t* cfull = aempty + kWqAStages;
+  uint64_t* xfull = reinterpret_cast<uint64_t*>(sStg + kWqEpiWarps * kStgWarpBytes);
+  uint64_t* xempty = xfull + kWqXStages;
+  uint64_t* cfull = xempty + kWqXStages;
   uint64_t* cempty = cfull + kWqMaxCStages;
-  uint64_t* bfull = cempty + kWqMaxCStages;
-  uint64_t* bempty = bfull + kWqBStages;
-  uint64_t* acc_full = bempty + kWqBStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* tfull = cempty + kWqMaxCStages;
+  uint64_t* tempty = tfull + kWqTStages;
+  uint64_t* acc_full = tempty + kWqTStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
   uint64_t* tile_full = drain + 1;
   uint64_t* tile_empty = tile_full + kTileRing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_empty + kTileRing);
@@ -197,22 +316,20 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
   constexpr int kCopy0 = kConv0 + kWqConvWarps;    // first weight-block issuer warp
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kWqAStages; ++s) {
-      mbar_init(&afull[s], 1);
-      mbar_init(&aempty[s], 1);  // the MMAs have read the A rows
+    for (int s = 0; s < kWqXStages; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);  // the MMAs have read the token rows
     }
     for (int s = 0; s < kCStages; ++s) {
       mbar_init(&cfull[s], kWqCopyWarps);   // one arrival (with its bytes) per block issuer
       mbar_init(&cempty[s], kWqConvWarps);  // every converter warp has read the codes
     }
-    for (int b = 0; b < kWqBStages; ++b) {
-      mbar_init(&bfull[b], kWqConvWarps);
-      mbar_init(&bempty[b], 1);
+    for (int t = 0; t < kWqTStages; ++t) {
+      mbar_init(&tfull[t], kWqConvWarps);   // the stage's weights are in TMEM
+      mbar_init(&tempty[t], 1);             // the MMAs have read them
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], kWqEpiWarps);
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kWqEpiWarps);
     mbar_init(drain, 1);
     for (int r = 0; r < kTileRing; ++r) {
       mbar_init(&tile_full[r], 1);
@@ -273,9 +390,12 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
     }
     return warp_wide ? __shfl_sync(0xffffffffu, ti, 0) : ti;
   };
+  // Weight block b of a tile exists: GATEUP always two (gate, up); DOWN the
+  // second only past the tile's first 128 columns.
+  auto has_block = [&](int b, int wn) -> bool { return GATEUP || b == 0 || wn > kBM; };
 
   if (warp == 0) {
-    // ------------------------------------------- producer (tiles, A rows)
+    // --------------------------------------- producer (tiles, token rows)
     int s = 0, issued = 0;
     uint32_t ph = 0;
     int rs = 0;
@@ -315,10 +435,10 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       for (int kb = 0; kb < kb_end; ++kb) {
         int waited = 1;
         if (lane == 0) {
-          waited = mbar_wait(&aempty[s], ph ^ 1, abort_flag, P.err);
+          waited = mbar_wait(&xempty[s], ph ^ 1, abort_flag, P.err);
           if (waited) {
-            mbar_arrive_expect_tx(&afull[s], a_small ? kASmallBytes : kAStageBytes);
-            tma_load_2d(sA + s * kAStageBytes, a_small ? &P.tmAs[p] : &P.tmA[p], &afull[s], kb * kBK, tile.row0);
+            mbar_arrive_expect_tx(&xfull[s], a_small ? kASmallBytes : kAStageBytes);
+            tma_load_2d(sX + s * kAStageBytes, a_small ? &P.tmAs[p] : &P.tmA[p], &xfull[s], kb * kBK, tile.row0);
           }
         }
         if (!__shfl_sync(0xffffffffu, waited, 0)) {
@@ -326,7 +446,7 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
           break;
         }
         ++issued;
-        if (++s == kWqAStages) {
+        if (++s == kWqXStages) {
           s = 0;
           ph ^= 1;
         }
@@ -335,12 +455,12 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       ti = __shfl_sync(0xffffffffu, next, 0);
     }
     __syncwarp();
-    if (lane == 0 && *abort_flag) drain_ring(afull, kWqAStages, s, ph, issued);
+    if (lane == 0 && *abort_flag) drain_ring(xfull, kWqXStages, s, ph, issued);
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------- MMA issuer
-      int s = 0, b = 0, acc = 0;
-      uint32_t ph = 0, bph = 0, acc_ph = 0;
+      int s = 0, t = 0;
+      uint32_t ph = 0, tph = 0, acc_ph = 0;
       bool any = false;
       int rs = 0;
       uint32_t rph = 0;
@@ -351,46 +471,43 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
         const int p = tile.pg >> 16;
         if (p >= P.nprob) break;
         const WqProblem& pr = P.prob[p];
-        const int wn = wq_tile_cols<GATEUP>(pr, tile.n0);
-        const uint32_t idesc = idesc_bf16_m128(GATEUP ? 2 * wn : wn, 0);  // B K-major
+        const bool two = has_block(1, wq_tile_cols<GATEUP>(pr, tile.n0));
+        const uint32_t idesc = idesc_bf16_m128((tile.rows + 15) & ~15, 0);  // N = the rows; B K-major
         const int kb_end = pr.K / kBK;
-        if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag, P.err)) break;
+        if (!mbar_wait(acc_empty, acc_ph ^ 1, abort_flag, P.err)) break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + acc * kAccCols;
         bool ok = true;
         for (int kb = 0; kb < kb_end; ++kb) {
-          if (!mbar_wait(&afull[s], ph, abort_flag, P.err) || !mbar_wait(&bfull[b], bph, abort_flag, P.err)) {
+          if (!mbar_wait(&xfull[s], ph, abort_flag, P.err) || !mbar_wait(&tfull[t], tph, abort_flag, P.err)) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_addr = smem_u32(sA + s * kAStageBytes);
-          const uint32_t b_addr = smem_u32(sB + b * kWqBStage);
+          const uint32_t x_addr = smem_u32(sX + s * kAStageBytes);
+          const uint32_t a0 = tmem_base + kWqTCol0 + t * kWqTStageCols;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            // both operands K-major, rows of 128 B, 8-row groups 1024 B apart; +32 B per 16 K
-            const uint64_t ad = sdesc_sw128(a_addr + k * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_addr + k * 32, 16, 1024);
-            umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            // token rows: K-major, rows of 128 B, 8-row groups 1024 B apart; +32 B per 16 K;
+            // weights in TMEM: 16 bf16 of K in 8 columns
+            const uint64_t bd = sdesc_sw128(x_addr + k * 32, 16, 1024);
+            umma_f16_tmem_a(tmem_base, a0 + 8 * k, bd, idesc, (kb | k) != 0);
+            if (two) umma_f16_tmem_a(tmem_base + kWqDCols, a0 + 32 + 8 * k, bd, idesc, (kb | k) != 0);
           }
           any = true;
-          umma_commit(&aempty[s]);  // A of this stage read
-          umma_commit(&bempty[b]);  // decoded weights read
-          if (++s == kWqAStages) {
+          umma_commit(&xempty[s]);  // token rows of this stage read
+          umma_commit(&tempty[t]);  // decoded weights read
+          if (++s == kWqXStages) {
             s = 0;
             ph ^= 1;
           }
-          if (++b == kWqBStages) {
-            b = 0;
-            bph ^= 1;
+          if (++t == kWqTStages) {
+            t = 0;
+            tph ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(&acc_full[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          acc_ph ^= 1;
-        }
+        umma_commit(acc_full);
+        acc_ph ^= 1;
       }
       if (any) {
         umma_commit(drain);
@@ -415,8 +532,7 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
         if (!tile_ok(tile)) break;  // the producer reports it
         const int p = tile.pg >> 16, g = tile.pg & 0xFFFF;
         const WqProblem& pr = P.prob[p];
-        const int wn = wq_tile_cols<GATEUP>(pr, tile.n0);
-        const bool mine = GATEUP || q == 0 || wn > 128;
+        const bool mine = has_block(q, wq_tile_cols<GATEUP>(pr, tile.n0));
         const int nb = (pr.N + 127) / 128, kbs = pr.K / kBK;
         const uint8_t* w = (GATEUP && q) ? pr.w1 : pr.w0;
         const int row_blk = (tile.n0 >> 7) + (GATEUP ? 0 : q);
@@ -445,12 +561,14 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
     }
   } else if (warp >= kConv0) {
     // ------------------------------------------------------- converters
-    // Item i of a stage: weight row r = i / 8 (B row: GATEUP gate rows
-    // 0..wn-1 then up rows, DOWN output columns), 16-byte piece c = i % 8
-    // (K 8c..8c+7 of the stage's 64).
-    const int ct = threadIdx.x - 32 * kConv0;
-    int s = 0, b = 0;
-    uint32_t ph = 0, bph = 0;
+    // Warp kConv0 + 4 b + j: weight block b, rows 32 q .. 32 q + 31 with
+    // q = warp % 4 (the TMEM lane quarter this warp may write), one row per
+    // thread: its 64 codes -> 32 bf16x2 columns of TMEM lane 32 q + lane.
+    const int cb = (warp - kConv0) >> 2;  // the block
+    const int r = (warp & 3) * 32 + lane;  // the row within it
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int s = 0, t = 0;
+    uint32_t ph = 0, tph = 0;
     int rs = 0;
     uint32_t rph = 0;
     while (true) {
@@ -459,103 +577,45 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       const Tile tile = P.tiles[ti];
       if (!tile_ok(tile)) break;
       const WqProblem& pr = P.prob[tile.pg >> 16];
-      const int wn = wq_tile_cols<GATEUP>(pr, tile.n0);
-      const int rows_b = GATEUP ? 2 * wn : wn;
+      const bool mine = has_block(cb, wq_tile_cols<GATEUP>(pr, tile.n0));
       const int kb_end = pr.K / kBK;
       bool ok = true;
       for (int kb = 0; kb < kb_end; ++kb) {
         const bool got =
-            mbar_wait(&cfull[s], ph, abort_flag, P.err) && mbar_wait(&bempty[b], bph ^ 1, abort_flag, P.err);
+            mbar_wait(&cfull[s], ph, abort_flag, P.err) && mbar_wait(&tempty[t], tph ^ 1, abort_flag, P.err);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
-        const uint8_t* cs = sC + s * kCS;
-        uint8_t* bs = sB + b * kWqBStage;
-        // A thread's (up to) kIt items of the stage: all code loads first, then
-        // the decodes, then the stores, so that the shared-memory latencies of
-        // the items overlap instead of adding up.
-        constexpr int kIt = 256 * 8 / kWqConvThreads;
-        const int n_items = rows_b * 8;
-        uint32_t w0[kIt], w1[kIt];
-        float dsc[kIt];
-#pragma unroll
-        for (int j = 0; j < kIt; ++j) {
-          const int i = ct + j * kWqConvThreads;
-          if (i >= n_items) continue;
-          const int r = i >> 3, c = i & 7;
-          // which copied block, and which of its rows, holds B row r
-          const int blk = GATEUP ? (r >= wn) : (r >> 7);
-          const int sr = GATEUP ? (r >= wn ? r - wn : r) : (r & 127);
-          const uint8_t* src = cs + blk * kBlk;
-          if (FMT == kWfSfp8) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(src + sr * 64 + 8 * c);
-            w0[j] = raw.x;
-            w1[j] = raw.y;
-          } else {
-            w0[j] = *reinterpret_cast<const uint32_t*>(src + sr * 32 + 4 * c);
-            dsc[j] = __half2float(*reinterpret_cast<const __half*>(src + 4096 + sr * 4 + 2 * (c >> 2)));
-          }
-        }
+        uint32_t v[32];
+        if (mine) wq_decode_row<FMT>(sC + s * kCS + cb * kBlk, r, v);
         __syncwarp();
         if (lane == 0) mbar_arrive(&cempty[s]);  // this warp is done with the stage's codes
-        uint4 o[kIt];
-#pragma unroll
-        for (int j = 0; j < kIt; ++j) {
-          const int i = ct + j * kWqConvThreads;
-          if (i >= n_items) continue;
-          uint32_t v[4];
-          if (FMT == kWfSfp8) {
-            // two codes per 32-bit word (one per 16-bit half), decoded together
-            v[0] = sfp8x2_to_bf16x2(__byte_perm(w0[j], 0u, 0x4140));
-            v[1] = sfp8x2_to_bf16x2(__byte_perm(w0[j], 0u, 0x4342));
-            v[2] = sfp8x2_to_bf16x2(__byte_perm(w1[j], 0u, 0x4140));
-            v[3] = sfp8x2_to_bf16x2(__byte_perm(w1[j], 0u, 0x4342));
-          } else {
-            // A nibble q at bit 8 (12) of a word, or'ed into the mantissa of
-            // 1.0, is the float f = 1 + q 2^-15 (1 + q 2^-11); one fma
-            // f A + B with A = d 2^15, B = -d (2^15 + 8) (2^11 for bit 12)
-            // gives (q - 8) d: A and B are exact (at most 13 x 11 significant
-            // bits), and so is (q - 8) d (4 x 11), so the fma's one rounding
-            // leaves it exact; then one rounding to bf16.
-            const float d = dsc[j];
-            const float a8 = __fmul_rn(d, 32768.0f), b8 = __fmul_rn(d, -32776.0f);
-            const float a12 = __fmul_rn(d, 2048.0f), b12 = __fmul_rn(d, -2056.0f);
-            const uint32_t x[4] = {w0[j] << 8, w0[j], w0[j] >> 8, w0[j] >> 16};  // elements 2qq, 2qq + 1 at bits 8, 12
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              const float lo = __uint_as_float((x[qq] & 0x00000F00u) | 0x3F800000u);
-              const float hi = __uint_as_float((x[qq] & 0x0000F000u) | 0x3F800000u);
-              v[qq] = pack_bf16x2(__fmaf_rn(lo, a8, b8), __fmaf_rn(hi, a12, b12));
-            }
-          }
-          o[j] = make_uint4(v[0], v[1], v[2], v[3]);
+        if (mine) {
+          tc_fence_after_sync();
+          tmem_st_32x32b_x32(tmem_base + lane_off + kWqTCol0 + t * kWqTStageCols + 32 * cb, v);
+          tmem_st_wait_all();
         }
-#pragma unroll
-        for (int j = 0; j < kIt; ++j) {
-          const int i = ct + j * kWqConvThreads;
-          if (i >= n_items) continue;
-          const int r = i >> 3, c = i & 7;
-          *reinterpret_cast<uint4*>(bs + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = o[j];
-        }
-        fence_proxy_async_smem();  // the MMA reads these bytes through the async proxy
+        tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bfull[b]);
+        if (lane == 0) mbar_arrive(&tfull[t]);
         if (++s == kCStages) {
           s = 0;
           ph ^= 1;
         }
-        if (++b == kWqBStages) {
-          b = 0;
-          bph ^= 1;
+        if (++t == kWqTStages) {
+          t = 0;
+          tph ^= 1;
         }
       }
       if (!ok) break;
     }
   } else {
     // ----------------------------------------------------------- epilogue
+    // lane = weight column 32 quarter + lane of D0 (block 0) and D1 (block 1);
+    // TMEM column j = the tile's row j. Stores transposed through the warp's
+    // staging buffer.
     const int quarter = warp & 3;
-    int acc = 0;
     uint32_t acc_ph = 0;
     int rs = 0;
     uint32_t rph = 0;
@@ -568,64 +628,55 @@ __global__ void __launch_bounds__(kWqThreads, 1) wq_gemm_kernel(const __grid_con
       if (p >= P.nprob) break;
       const WqProblem& pr = P.prob[p];
       const int wn = wq_tile_cols<GATEUP>(pr, tile.n0);
-      const bool ready = mbar_wait(&acc_full[acc], acc_ph, abort_flag, P.err);
+      const bool ready = mbar_wait(acc_full, acc_ph, abort_flag, P.err);
       __syncwarp();
       if (!ready) break;
+      acc_ph ^= 1;
       tc_fence_after_sync();
-      const uint32_t tbase = tmem_base + acc * kAccCols + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int rows_valid = tile.rows - quarter * 32;
-      const size_t wrow = static_cast<size_t>(tile.row0 + quarter * 32);
+      const uint32_t t0 = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
       const float sc0 = (FMT == kWfSfp8 && pr.s0) ? pr.s0[g] : 1.0f;
       const float sc1 = (FMT == kWfSfp8 && pr.s1) ? pr.s1[g] : 1.0f;
-      if (rows_valid > 0) {
-        if (GATEUP) {
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out) + wrow * pr.ldo + tile.n0;
-          for (int j = 0; j < wn; j += 32) {
+      const int n_tok = tile.rows;
+      if (GATEUP) {
+        // gate in D0, up in D1, both for columns n0 + 32 quarter + lane
+        if (quarter * 32 < wn) {
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(pr.out) + static_cast<size_t>(tile.row0) * pr.ldo +
+                               tile.n0 + quarter * 32;
+          for (int j = 0; j < n_tok; j += 32) {
             uint32_t gt[32], up[32];
-            tmem_ld_32x32b_x32(tbase + j, gt);
-            tmem_ld_32x32b_x32(tbase + wn + j, up);
+            tmem_ld_32x32b_x32(t0 + j, gt);
+            tmem_ld_32x32b_x32(t0 + kWqDCols + j, up);
             tmem_ld_wait();
-            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = gelu_tanh(__uint_as_float(gt[2 * i]) * sc0) * (__uint_as_float(up[2 * i]) * sc1);
-              const float h1 =
-                  gelu_tanh(__uint_as_float(gt[2 * i + 1]) * sc0) * (__uint_as_float(up[2 * i + 1]) * sc1);
-              pk[i] = pack_bf16x2(h0, h1);
-            }
-            store_rows_bf16x32(stg, pk, lane, out + j, pr.ldo, rows_valid);
+            for (int i = 0; i < 32; ++i)
+              gt[i] = __float_as_uint(gelu_tanh(__uint_as_float(gt[i]) * sc0) * (__uint_as_float(up[i]) * sc1));
+            store_cols_bf16x32(stg, gt, lane, out + static_cast<size_t>(j) * pr.ldo, pr.ldo, n_tok - j);
           }
-        } else {
-          for (int j = 0; j < wn; j += 32) {
+        }
+      } else {
+        // D0: columns n0 + 32 quarter + lane, D1: the same plus 128
+        for (int b = 0; b < 2; ++b) {
+          const int c = b * kBM + quarter * 32;
+          if (c >= wn) continue;
+          for (int j = 0; j < n_tok; j += 32) {
             uint32_t a[32];
-            tmem_ld_32x32b_x32(tbase + j, a);
+            tmem_ld_32x32b_x32(t0 + b * kWqDCols + j, a);
             tmem_ld_wait();
             if (FMT == kWfSfp8) {
 #pragma unroll
               for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * sc0);
             }
-            if (pr.out_f32) {
-              store_rows_f32x32(stg, a, lane, reinterpret_cast<float*>(pr.out) + wrow * pr.ldo + tile.n0 + j, pr.ldo,
-                                rows_valid);
-            } else {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
-              store_rows_bf16x32(stg, pk, lane,
-                                 reinterpret_cast<__nv_bfloat16*>(pr.out) + wrow * pr.ldo + tile.n0 + j, pr.ldo,
-                                 rows_valid);
-            }
+            const size_t off = static_cast<size_t>(tile.row0 + j) * pr.ldo + tile.n0 + c;
+            if (pr.out_f32)
+              store_cols_f32x32(stg, a, lane, reinterpret_cast<float*>(pr.out) + off, pr.ldo, n_tok - j);
+            else
+              store_cols_bf16x32(stg, a, lane, reinterpret_cast<__nv_bfloat16*>(pr.out) + off, pr.ldo, n_tok - j);
           }
         }
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_ph ^= 1;
-      }
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
 
@@ -702,9 +753,10 @@ __global__ void wq_quant_kernel(const __nv_bfloat16* __restrict__ w, int K, int 
       for (int b = 0; b < 4; ++b) wd |= static_cast<uint32_t>(sfp8_encode_dev(__fdiv_rn(x[4 * j + b], sc))) << (8 * b);
       words[j] = wd;
     }
-    uint4* dst = reinterpret_cast<uint4*>(blk + r * 64);
+    uint4* dst = reinterpret_cast<uint4*>(blk + r * 64);  // piece j at position j ^ ((r >> 1) & 3)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
+    for (int j = 0; j < 4; ++j)
+      dst[j ^ ((r >> 1) & 3)] = make_uint4(words[4 * j], words[4 * j + 1], words[4 * j + 2], words[4 * j + 3]);
   } else {
     uint32_t words[8];
     __half scales[2];
@@ -730,9 +782,9 @@ __global__ void wq_quant_kernel(const __nv_bfloat16* __restrict__ w, int K, int 
         words[4 * hb + j] = wd;
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(blk + r * 32);
-    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    uint4* dst = reinterpret_cast<uint4*>(blk + r * 32);  // piece j at position j ^ ((r >> 2) & 1)
+    dst[(r >> 2) & 1] = make_uint4(words[0], words[1], words[2], words[3]);
+    dst[((r >> 2) & 1) ^ 1] = make_uint4(words[4], words[5], words[6], words[7]);
     __half2 hs;
     hs.x = scales[0];
     hs.y = scales[1];

@@ -30,15 +30,23 @@ def _gpu():
     require_gpu()
 
 
+def _unswizzle(rows: np.ndarray, shift: int, mask: int) -> np.ndarray:
+    """[..., 128 rows, pieces, 16 B] stored with piece j of row r at position j ^ ((r >> shift) & mask)
+    -> pieces in K order."""
+    r = np.arange(128)[:, None]
+    j = np.arange(rows.shape[-2])[None, :]
+    return rows[..., r, j ^ ((r >> shift) & mask), :]
+
+
 def decode_layout(q: np.ndarray, fmt: str, G: int, K: int, N: int):
     """The library's blocks -> (codes [G][N][K], Q4_0 scales [G][N][K/32] or None, padding rows)."""
     nb, kb = (N + 127) // 128, K // 64
     if fmt == "sfp8":
-        blk = q.reshape(G, nb, kb, 128, 64)
+        blk = _unswizzle(q.reshape(G, nb, kb, 128, 4, 16), 1, 3).reshape(G, nb, kb, 128, 64)
         codes = blk.transpose(0, 1, 3, 2, 4).reshape(G, nb * 128, K)
         return codes[:, :N], None, codes[:, N:]
     blk = q.reshape(G, nb, kb, 4608)
-    cb = blk[..., :4096].reshape(G, nb, kb, 128, 32)
+    cb = _unswizzle(blk[..., :4096].reshape(G, nb, kb, 128, 2, 16), 2, 1).reshape(G, nb, kb, 128, 32)
     nib = np.empty((G, nb, kb, 128, 64), np.uint8)
     nib[..., 0::2] = cb & 0xF
     nib[..., 1::2] = cb >> 4
