@@ -449,25 +449,47 @@ def run_ours(args, world, rank, local):
     agg = res_t["agg"]
     stream = torch.cuda.current_stream()
 
-    # ---- end to end: host buffers through the C ABI, copies inside the timed region
+    # ---- end to end: host buffers through the C ABI, copies inside the timed
+    # region. Two streams, each with its own device buffers and workspace,
+    # take alternate batches, as a serving loop would: one batch's copies
+    # overlap the other's kernels, and every batch's host-to-device and
+    # device-to-host copies stay inside the timed region.
+    from mixture_experts_transformer_b200 import block as blk
+    from mixture_experts_transformer_b200 import inputs as inp
+
     x_host = x.cpu().pin_memory()
-    out_host = torch.empty((T, D), dtype=torch.bfloat16).pin_memory()
+    lanes = []
     for _ in range(2):
-        B.check(B.moe_block_forward_hostio(p, x_host, out_host, stream), "hostio")
+        xk, ok_ = torch.empty_like(x), torch.empty_like(out)
+        wsk, _ = blk.workspace_for(inp.GEMMA4_26B_A4B, T)
+        pk = B.make_params(T, xk, *dw.args(), ok_, router_bias=bias, workspace=wsk, **sandwich)
+        lanes.append((torch.cuda.Stream(), pk, torch.empty((T, D), dtype=torch.bfloat16).pin_memory(), xk, ok_, wsk))
+
+    def e2e_batch(i):
+        st, pk, oh = lanes[i % 2][:3]
+        B.check(B.moe_block_forward_hostio(pk, x_host, oh, st), "hostio")
+
+    for i in range(4):
+        e2e_batch(i)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(args.steps):
-        B.check(B.moe_block_forward_hostio(p, x_host, out_host, stream), "hostio")
+    for ln in lanes:
+        ln[0].wait_stream(stream)
+    for i in range(args.steps):
+        e2e_batch(i)
+    for ln in lanes:
+        stream.wait_stream(ln[0])
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = reduce_max(t0.elapsed_time(t1), world)
     barrier(world)
-    if not torch.equal(out_host, out.cpu()):
+    if not all(torch.equal(ln[2], out.cpu()) for ln in lanes):
         raise RuntimeError("host-buffer path disagrees with the device path")
+    del lanes
     ws_bytes = res_t["ws"].numel()
     del res_t["ws"], res_t["x"], res_t["out"], res_t["p"]
 
@@ -510,6 +532,7 @@ def run_ours(args, world, rank, local):
             "unit": "tokens/s",
             "h2d_bytes_per_step": T * D * 2,
             "d2h_bytes_per_step": T * D * 2,
+            "overlap": "two streams take alternate batches through moe_block_forward_hostio",
         },
         "clocks": res_t["clocks"],
         "workspace_bytes": ws_bytes,
@@ -1171,7 +1194,7 @@ def run_wq(args, world, rank, local):
             "peak_source": f"{peaks['source']} hbm_gbs",
             "unit": "GB/s",
             "frac": byts / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "traffic": None,
+            "traffic": ncu_traffic(dominant, args.workload),
             "algorithmic_bytes": byts,
             "kernel_ms": dom_ms,
         },

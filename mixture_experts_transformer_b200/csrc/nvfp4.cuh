@@ -649,9 +649,9 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
       const bool valid = r < tile.rows;
       const int grow = tile.row0 + r;
       // Column chunks of 32: j = half * 32 + 64 c (c = 0..3 while j < wn).
-      // Gate|up brings all of this thread's accumulator columns (gate and up
-      // of chunks 0, 1) into registers and hands TMEM back at once, so the
-      // next tile's MMAs overlap the math and stores below. Down holds 4
+      // Gate|up brings this thread's accumulator columns (gate and up of
+      // chunks 0, 1) into registers and hands TMEM back, so the next tile's
+      // MMAs overlap the quantisation and stores below. Down holds 4
       // chunks: chunks 0, 1 are converted and stored first, then chunks 2, 3
       // are loaded and TMEM handed back (64 values in registers at a time).
       uint32_t acc[4][32];
@@ -666,40 +666,47 @@ __global__ void __launch_bounds__(f4_threads<GATEUP>(), 1) fp4_gemm_kernel(const
         }
       };
       if (GATEUP) {
+        // Chunk 0 (gate and up columns j0 = 32 half) is loaded, turned into h
+        // and quantised before chunk 1 (j0 + 64) is loaded and TMEM handed
+        // back: at most 64 accumulator values live at a time, no spills.
+        const float ag = 1.0f / (pr.ga * pr.gb0[g]);
+        const float au = 1.0f / (pr.ga * pr.gb1[g]);
+        uint8_t* q = reinterpret_cast<uint8_t*>(pr.out) + static_cast<size_t>(grow) * (pr.N / 2);
+        uint4 qc[2];
+        uint32_t sc[2][2];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int j = half * 32 + 64 * c;
           if (j < wn) {
-            tmem_ld_32x32b_x32(tbase + j, acc[c]);
-            tmem_ld_32x32b_x32(tbase + 128 + j, acc[2 + c]);
+            tmem_ld_32x32b_x32(tbase + j, acc[0]);
+            tmem_ld_32x32b_x32(tbase + 128 + j, acc[1]);
           }
-        }
-        release_acc();
-      }
-      if (GATEUP) {
-        const float ag = 1.0f / (pr.ga * pr.gb0[g]);
-        const float au = 1.0f / (pr.ga * pr.gb1[g]);
-        uint8_t* q = reinterpret_cast<uint8_t*>(pr.out) + static_cast<size_t>(grow) * (pr.N / 2);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int j = half * 32 + 64 * c;
+          if (c == 1) {
+            release_acc();
+          } else {
+            tmem_ld_wait();
+          }
           if (j >= wn) continue;
           uint2 codes[2];
-          uint32_t sc[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             float v[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              v[i] = gelu_tanh(__uint_as_float(acc[c][16 * h + i]) * ag) *
-                     (__uint_as_float(acc[2 + c][16 * h + i]) * au);
-            sc[h] = nvfp4_group(v, pr.g_out, &codes[h]);
+              v[i] = gelu_tanh(__uint_as_float(acc[0][16 * h + i]) * ag) * (__uint_as_float(acc[1][16 * h + i]) * au);
+            sc[c][h] = nvfp4_group(v, pr.g_out, &codes[h]);
           }
-          if (valid) {
-            *reinterpret_cast<uint4*>(q + (tile.n0 + j) / 2) = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+          qc[c] = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+        }
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int j = half * 32 + 64 * c;
+            if (j >= wn) continue;
+            *reinterpret_cast<uint4*>(q + (tile.n0 + j) / 2) = qc[c];
             const int c16 = (tile.n0 + j) / 16;
-            pr.out_sf[sf_offset(grow, c16, pr.N / 64)] = static_cast<uint8_t>(sc[0]);
-            pr.out_sf[sf_offset(grow, c16 + 1, pr.N / 64)] = static_cast<uint8_t>(sc[1]);
+            pr.out_sf[sf_offset(grow, c16, pr.N / 64)] = static_cast<uint8_t>(sc[c][0]);
+            pr.out_sf[sf_offset(grow, c16 + 1, pr.N / 64)] = static_cast<uint8_t>(sc[c][1]);
           }
         }
       } else {
