@@ -135,28 +135,26 @@ __host__ __device__ inline uint16_t sfp8_bf16_bits(uint32_t code) {
   return static_cast<uint16_t>(bits | ((code & 0x80u) << 8));
 }
 
-// Bytes 0 and 2 of x, each replaced by copies of its top bit, in both bytes
-// of their 16-bit halves: prmt's sign-replicating selectors (CUDA's
-// __byte_perm keeps only the byte-select bits of a selector).
-__device__ __forceinline__ uint32_t replicate_top_bits_b02(uint32_t x) {
+// Per 16-bit half, the smaller of a and b (unsigned).
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
-  asm("prmt.b32 %0, %1, 0, 0xAA88;" : "=r"(r) : "r"(x));
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
 // Two SFP8 codes, in bytes 0 and 2 of v (bytes 1 and 3 are ignored), to two
-// bf16 bit patterns: m >= 64 -> 0x3800 + 16 m, 1 <= m < 64 -> 0x3400 + 32 m,
-// m = 0 -> 0, sign to bit 15. Both candidates are computed in packed 16-bit
-// lanes and selected by per-lane masks spread from one bit of each code
-// (bit 6: m >= 64; the carry of m + 127 into bit 7: m != 0). Equal to
-// sfp8_bf16_bits for all 2^16 code pairs.
+// bf16 bit patterns, in packed 16-bit lanes: m >= 64 -> 0x3800 + 16 m,
+// 1 <= m < 64 -> 0x3400 + 32 m, m = 0 -> 0, sign to bit 15. The two linear
+// pieces meet at m = 64 (0x3C00); below it 0x3400 + 32 m is the smaller, above
+// it 0x3800 + 16 m, so their minimum is the value, and a third term, 0 for
+// m = 0 and 0x7FFF otherwise, makes the minimum 0 for the zero code. Mostly
+// multiply-adds; equal to sfp8_bf16_bits for all 2^16 code pairs.
 __device__ __forceinline__ uint32_t sfp8x2_to_bf16x2(uint32_t v) {
   const uint32_t m = v & 0x007F007Fu;
   const uint32_t lg = m * 16u + 0x38003800u;
   const uint32_t sm = m * 32u + 0x34003400u;
-  const uint32_t big = replicate_top_bits_b02(v << 1);
-  const uint32_t nz = replicate_top_bits_b02(m + 0x007F007Fu);
-  return (((lg & big) | (sm & ~big)) & nz) | ((v << 8) & 0x80008000u);
+  const uint32_t z = min_u16x2(m, 0x00010001u) * 0x7FFFu;
+  return (v & 0x00800080u) * 256u + min_u16x2(min_u16x2(lg, sm), z);
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
