@@ -445,8 +445,8 @@ def run_ours(args, world, rank, local):
             "residual": True,
         }
     # ---- the metric's prefill half: the T = 4096 block, timed the same way,
-    # first (the tensor-bound half draws the most power; timed second it met
-    # the power cap left by the decode half's runs more often)
+    # first: the tensor-bound half draws the most power, and timed after the
+    # decode half's passes it ran at a lower power-capped clock
     prefill = None
     if args.workload == "decode" and not args.no_prefill:
         wp = WORKLOADS["prefill"]
@@ -454,6 +454,9 @@ def run_ours(args, world, rank, local):
         del res_p["ws"], res_p["x"], res_p["out"], res_p["p"]
         prefill = res_p
         torch.cuda.empty_cache()
+        # let the power limiter's average settle before the decode half, as
+        # between two separate runs (timing is on the device in both halves)
+        time.sleep(3.0)
 
     res_t = time_block(B, dw, T, bias, args.steps, args.warmup, world, local, sandwich, rank)
     x, out, p = res_t["x"], res_t["out"], res_t["p"]
