@@ -486,11 +486,15 @@ moe_status enqueue_route(const Dims& d, const Layout& L, uint8_t* ws, const void
   }
   LaunchScope ls_(kKRouterTopk, st);
   const int tk_blocks = (d.T + kTopkWarps - 1) / kTopkWarps;
+  // large batches: two tokens per warp (E <= 128, k <= 16)
+  const bool tk_pair = d.E <= 128 && d.k <= 16 && d.T >= 1024;
   const cudaError_t le_ =
-      L.nsplit > 8 ? launch_k(router_topk_kernel<true>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
-                              L.nsplit, d.k, idx, w, masks, logits_out)
-                   : launch_k(router_topk_kernel<false>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
-                              L.nsplit, d.k, idx, w, masks, logits_out);
+      tk_pair ? launch_k(router_topk_pair_kernel, (d.T + 2 * kTopkWarps - 1) / (2 * kTopkWarps), kTopkWarps * 32, 0,
+                         st, partial, bias, d.T, d.E, L.nsplit, d.k, idx, w, masks, logits_out)
+      : L.nsplit > 8 ? launch_k(router_topk_kernel<true>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
+                                L.nsplit, d.k, idx, w, masks, logits_out)
+                     : launch_k(router_topk_kernel<false>, tk_blocks, kTopkWarps * 32, 0, st, partial, bias, d.T, d.E,
+                                L.nsplit, d.k, idx, w, masks, logits_out);
   return ls_.done(le_);
 }
 
@@ -506,7 +510,7 @@ moe_status enqueue_permute(const Dims& d, const Layout& L, uint8_t* ws, const in
   const bool pairs = allow_pairs && pair_sm(d, s);
   {
     LaunchScope ls_(kKRouteScan, st);
-    const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
+    const cudaError_t le_ = launch_k(route_scan_kernel, kScanCtas, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
                                      reinterpret_cast<TileCounts*>(ws + L.counts), 0, 256, 128,
@@ -782,7 +786,7 @@ moe_status enqueue_block_fp4(const moe_nvfp4_params* p, const Dims& d, const Fp4
   MOE_TRY(enqueue_route(d, L, ws, p->x, p->w_router, p->router_bias, idx, w, st));
   {
     LaunchScope ls_(kKRouteScan, st);
-    const cudaError_t le_ = launch_k(route_scan_kernel, 1, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
+    const cudaError_t le_ = launch_k(route_scan_kernel, kScanCtas, kScanThreads, 0, st, masks, L.nchunks, d.T, d.E, d.F, d.S,
                                      d.D, base, cnt, off, reinterpret_cast<Tile*>(ws + L.tiles_gu),
                                      reinterpret_cast<Tile*>(ws + L.tiles_dn),
                                      reinterpret_cast<TileCounts*>(ws + L.counts), 1, 256, 128, 0, 0, 0, d.E);

@@ -23,6 +23,9 @@ constexpr int kScanThreads = 1024;
 // row_of of a (token, slot) whose expert belongs to another expert shard
 constexpr int32_t kRowNotLocal = -1;
 constexpr int kScanSegs = kScanThreads / 128;
+// CTAs of the scan (each recomputes the offsets from the masks and emits a
+// share of the tiles and of base)
+constexpr int kScanCtas = 8;
 
 struct TileCounts {
   int32_t gateup;
@@ -48,8 +51,10 @@ __global__ void build_masks_kernel(const int32_t* __restrict__ idx, int T, int k
   }
 }
 
-// One CTA of 1024 threads: thread (e, seg) walks one eighth of the 32-token
-// chunks of expert e. Produces cnt, off, base[c][e] and the tile lists
+// kScanCtas CTAs of 1024 threads, each computing the same per-expert counts
+// and offsets (thread (e, seg) walks one eighth of the 32-token chunks of
+// expert e); CTA b then writes base[c][e] for the chunks of segment b and
+// every kScanCtas-th entry of the tile lists. Produces cnt, off, base and the tile lists
 // (gate|up tiles gu_cols output columns per projection, down tiles dn_cols wide):
 // shared-MLP tiles first (problem 1), then expert tiles (problem 0) expert by
 // expert, column tile, then row tile, so CTAs that run at the same time read
@@ -134,7 +139,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   // first routed row of expert e: packed (bf16 path) or padded to whole
   // 128-row tiles (NVFP4 path: every tile starts on a scale-atom boundary)
   const int row_base = padded ? s_mtoff[e] * kBM : s_off[e];
-  if (local) {
+  if (local && seg % gridDim.x == blockIdx.x) {
     int run = row_base + s_seg[seg][e];
 #pragma unroll 8
     for (int c = c0; c < c1; ++c) {
@@ -142,11 +147,15 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
       run += __popc(__ldg(masks + static_cast<size_t>(c) * E + e));
     }
   }
-  if (e < E && seg == 0) {
-    cnt_out[e] = c_e;
-    off_out[e] = s_off[e];
+  if (blockIdx.x == 0) {
+    if (e < E && seg == 0) {
+      cnt_out[e] = c_e;
+      off_out[e] = s_off[e];
+    }
+    if (threadIdx.x == 0) off_out[E] = s_off[E];
   }
-  if (threadIdx.x == 0) off_out[E] = s_off[E];
+  const int gt = blockIdx.x * kScanThreads + threadIdx.x;  // this thread's first list entry
+  const int gstride = gridDim.x * kScanThreads;
 
   // A tile takes one 128-row block, or (paired GEMM) two consecutive blocks of
   // the same expert and column tile. Gate|up tiles are gu_cols output columns
@@ -159,7 +168,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     const int* offs = pair ? s_ptoff : s_mtoff;
     const int pt_sh = (mt_sh + mstep - 1) / mstep;
     const int n_sh = ncol_sh * pt_sh;
-    for (int i = threadIdx.x; i < n_sh; i += kScanThreads) {
+    for (int i = gt; i < n_sh; i += gstride) {
       const int nt = i / pt_sh, m = (i % pt_sh) * mstep;
       const int r1 = pair ? max(0, min(kBM, T - (m + 1) * kBM)) : 0;
       tiles[i] = Tile{1 << 16, m * kBM, min(kBM, T - m * kBM), nt * cw, (m + 1) * kBM, r1, 0, 0};
@@ -167,7 +176,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
     // expert tiles, spread over all threads (one expert may own most of them):
     // flat index f -> expert by binary search over the tile-offset prefix
     const int n_e = offs[E] * ncol;
-    for (int f = threadIdx.x; f < n_e; f += kScanThreads) {
+    for (int f = gt; f < n_e; f += gstride) {
       int lo = 0, hi = E - 1;  // largest ex with offs[ex] * ncol <= f
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -187,7 +196,7 @@ __global__ void __launch_bounds__(kScanThreads) route_scan_kernel(const uint32_t
   };
   const int n_gu = emit(tiles_gu, pair_gu, (S + gu_cols - 1) / gu_cols, nt_gu, gu_cols);
   const int n_dn = emit(tiles_dn, pair_dn, (D + dn_cols - 1) / dn_cols, nt_dn, dn_cols);
-  if (threadIdx.x == 0) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     counts->gateup = n_gu;
     counts->down = n_dn;
     counts->next_gateup = 0;

@@ -52,8 +52,10 @@ def test_router_logits_against_oracle(T, skew):
     assert err.max() <= LOGIT_TOL, err.max()
 
 
-@pytest.mark.parametrize("T", [1, 7, 64, 257])
+@pytest.mark.parametrize("T", [1, 7, 64, 257, 1025, 2048])
 def test_route_gemma(T):
+    """Routing against the oracle; from T = 1024 the top-k takes two tokens per
+    warp (1025: the last warp's second half has no token)."""
     w = weights()
     dw = device_weights()
     x_bits = inputs.make_x(T, seed=11 + T)
@@ -67,11 +69,13 @@ def test_route_gemma(T):
     check_routing(logits, ref_idx, ref_w, to_np(idx), to_np(wt), 8)
 
 
-def test_route_ties_pick_lower_index():
+@pytest.mark.parametrize("T", [96, 1030])
+def test_route_ties_pick_lower_index(T):
     """Duplicated router columns give bitwise-equal fp32 logits on the GPU too;
-    the lower expert index must be selected first."""
+    the lower expert index must be selected first (one token per warp at
+    T = 96, two at T = 1030)."""
     rng = np.random.default_rng(3)
-    d, e, T = 256, 16, 96
+    d, e = 256, 16
     wr = inputs.f32_to_bf16_bits(rng.standard_normal((d, e)).astype(np.float32) * 0.1)
     wr[:, 9] = wr[:, 3]
     wr[:, 14] = wr[:, 3]
