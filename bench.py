@@ -3,7 +3,10 @@
 
 One "step" is one pass of the block (router, top-k, permutation, gate|up and
 down grouped GEMMs, shared MLP, combine) over one batch of T tokens, through
-the library's C ABI. Default workload: the decode-sized block, T = 64 tokens.
+the library's C ABI. Default workload: the decode-sized block, T = 64 tokens;
+on one GPU its line also carries the prefill-sized block (T = 4096, key
+"prefill", timed first) and the NVFP4 30-layer stack (T = 2048, key
+"nvfp4_stack", timed last), each measured the same way.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload decode|tiny|prefill|skewed]
   python bench.py --impl reference ...   # the CPU oracle on the same workload
@@ -96,6 +99,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="decode workload: skip the T=4096 prefill run that the default line carries")
+    ap.add_argument("--no-stack", action="store_true",
+                    help="decode workload: skip the NVFP4 30-layer stack run that the default line carries (one GPU)")
     ap.add_argument("--sandwich", action="store_true",
                     help="bf16 workloads: time the block with the pre/post-FFN RMSNorm sandwich and the residual add")
     ap.add_argument("--layers", type=int, default=None, help="nvfp4_stack depth (default 30)")
@@ -1235,6 +1240,17 @@ def main():
             res = run_wq(args, world, rank, local)
         else:
             res = run_ours(args, world, rank, local)
+            if args.workload == "decode" and world == 1 and not args.no_stack and not args.sandwich:
+                # the NVFP4 30-layer stack (T=2048), timed the same way, as a key of the default line
+                import copy
+
+                import torch
+
+                torch.cuda.empty_cache()
+                time.sleep(3.0)
+                sargs = copy.copy(args)
+                sargs.workload, sargs.no_cpu_baseline, sargs.layers = "nvfp4_stack", True, None
+                res["nvfp4_stack"] = run_stack(sargs, world, rank, local)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:
