@@ -568,8 +568,8 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
             map_3d(&gu.tmB1[0], p->wu, d.el, d.D, d.F) && map_2d(&gu.tmA[1], xin, d.T, d.D, kBM) &&
             map_3d(&gu.tmB0[1], p->sg, 1, d.D, d.S) && map_3d(&gu.tmB1[1], p->su, 1, d.D, d.S);
   if (!ok) return MOE_ERR_CUDA;
-  gu.prob[0] = GemmProblem{d.D, d.F, d.el, static_cast<int>(R), h, d.F, 0};
-  gu.prob[1] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
+  gu.prob[0] = GemmProblem{d.D, d.F, d.el, static_cast<int>(R), h, d.F, 0, 0};
+  gu.prob[1] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0, 0};
   gu.nprob = 2;
   gu.stream_weights = stream_weights(d) ? 1 : 0;
   gu.a_wide = paired_gateup(d) ? 1 : 0;
@@ -598,8 +598,8 @@ moe_status enqueue_block(const moe_params* p, const Dims& d, const Layout& L, ui
   if (!ok) return MOE_ERR_CUDA;
   dn.tmB1[0] = dn.tmB0[0];
   dn.tmB1[1] = dn.tmB0[1];
-  dn.prob[0] = GemmProblem{d.F, d.D, d.el, static_cast<int>(R), y, d.D, 0};
-  dn.prob[1] = GemmProblem{d.S, d.D, 1, d.T, sbuf, d.D, 1};
+  dn.prob[0] = GemmProblem{d.F, d.D, d.el, static_cast<int>(R), y, d.D, 0, 0};
+  dn.prob[1] = GemmProblem{d.S, d.D, 1, d.T, sbuf, d.D, 1, 0};
   dn.nprob = 2;
   dn.stream_weights = gu.stream_weights;
   // 256-column tiles: 4 chunks per copy on one SM, 2 per CTA on SM pairs
@@ -1100,7 +1100,7 @@ moe_status enqueue_dense(const moe_dense_params* p, const DenseDims& d, const De
   if (!map_2d(&gu.tmA[0], p->x, d.T, d.D, kBM) || !map_3d(&gu.tmB0[0], p->wg, 1, d.D, d.S) ||
       !map_3d(&gu.tmB1[0], p->wu, 1, d.D, d.S))
     return MOE_ERR_CUDA;
-  gu.prob[0] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0};
+  gu.prob[0] = GemmProblem{d.D, d.S, 1, d.T, hs, d.S, 0, 0};
   gu.nprob = 1;
   gu.stream_weights = d.T <= kBM ? 1 : 0;  // one row block reads each weight tile once
   gu.a_wide = pairs ? 1 : 0;
